@@ -1,0 +1,46 @@
+"""Parity helpers shared by the tests: the tolerance the grouped matmuls
+must meet against the oracle, and checks that a comparison is not vacuous."""
+from __future__ import annotations
+
+import numpy as np
+
+
+def bf16_bits_to_f64(h) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def bf16_ulp(v) -> np.ndarray:
+    """Spacing of bf16 numbers at |v| (8 significant bits; subnormal floor)."""
+    a = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.exp2(e - 7)
+
+
+def row_tolerance(oracle_f64: np.ndarray, rel: float = 1e-2) -> np.ndarray:
+    """|gpu - oracle| <= rel * rms(oracle row) + 1 bf16 ulp(oracle value),
+    elementwise; rows are the last axis."""
+    o = np.asarray(oracle_f64, np.float64)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True)) if o.shape[-1] else 0.0
+    return rel * rms + bf16_ulp(o)
+
+
+def check_rows(gpu_bf16_bits, oracle_f64, rel: float = 1e-2):
+    """Returns (ok, worst normalised error, number of elements compared).
+    Raises if nothing was compared (an empty comparison is not a pass)."""
+    g = bf16_bits_to_f64(gpu_bf16_bits)
+    o = np.asarray(oracle_f64, np.float64)
+    assert g.shape == o.shape, (g.shape, o.shape)
+    if o.size == 0:
+        raise AssertionError("empty comparison")
+    tol = row_tolerance(o, rel)
+    err = np.abs(g - o)
+    bad = ~(err <= tol)  # NaN counts as bad
+    worst = float(np.max(err / tol))
+    return (not bool(bad.any())), worst, int(o.size)
+
+
+def assert_rows_close(gpu_bf16_bits, oracle_f64, rel: float = 1e-2, what=""):
+    ok, worst, n = check_rows(gpu_bf16_bits, oracle_f64, rel)
+    assert ok, f"{what}: {n} elements, worst |err|/tol = {worst:.3g} (> 1)"
+    return worst
