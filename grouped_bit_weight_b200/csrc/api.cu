@@ -1,0 +1,253 @@
+// api.cu -- the extern "C" entry points declared in include/gbw.h: host-side
+// argument checks, the sm_100 check, the per-device error word and the
+// choice between the tensor-core GEMM and the bandwidth GEMV.
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace gbw {
+namespace {
+
+// GBW_DEVERR_* bits raised by the kernels of this library on this device.
+__device__ int g_err_word;
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices];
+int g_sms[kMaxDevices];
+int g_arch_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+
+thread_local char g_msg[256] = "";
+
+gbw_status launch_error(cudaError_t e) {
+  snprintf(g_msg, sizeof(g_msg), "CUDA error: %s", cudaGetErrorString(e));
+  return GBW_ERR_LAUNCH;
+}
+
+// Per-device state: architecture check, SM count and the device address of
+// the error word (resolved with the device current).
+gbw_status device_state(int** err, int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return launch_error(e);
+  if (dev < 0 || dev >= kMaxDevices) return GBW_ERR_ARCH;
+  if (g_arch_ok[dev] == 0) {
+    int major = 0, minor = 0, n = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (major != 10 || minor != 0) {
+      g_arch_ok[dev] = -1;
+    } else {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_err_word);
+      if (e != cudaSuccess) return launch_error(e);
+      g_err_ptr[dev] = static_cast<int*>(p);
+      g_sms[dev] = n;
+      g_arch_ok[dev] = 1;
+    }
+  }
+  if (g_arch_ok[dev] < 0) {
+    snprintf(g_msg, sizeof(g_msg), "device %d is not sm_100 (B200)", dev);
+    return GBW_ERR_ARCH;
+  }
+  *err = g_err_ptr[dev];
+  *sms = g_sms[dev];
+  return GBW_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+gbw_status fail(gbw_status s, const char* what) {
+  snprintf(g_msg, sizeof(g_msg), "%s", what);
+  return s;
+}
+
+gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
+                           const uint8_t* w, const void* scale, int32_t E,
+                           int64_t N, const int32_t* offsets,
+                           const int32_t* row_to_token, int64_t P,
+                           uint16_t* out, int32_t mode, void* stream) {
+  if (T < 0 || K <= 0 || N <= 0 || E < 1 || P < 0)
+    return fail(GBW_ERR_SHAPE, "need T >= 0, K > 0, N > 0, E >= 1, P >= 0");
+  if (f == Fmt::NF4 && K % 64) return fail(GBW_ERR_SHAPE, "NF4 needs K % 64 == 0");
+  if (f == Fmt::MXFP4 && K % 32) return fail(GBW_ERR_SHAPE, "MXFP4 needs K % 32 == 0");
+  if (N % 8) return fail(GBW_ERR_SHAPE, "N must be a multiple of 8");
+  if (K > (int64_t)1 << 30 || N > (int64_t)1 << 30 || P > INT32_MAX ||
+      T > INT32_MAX || (int64_t)E * N > INT32_MAX)
+    return fail(GBW_ERR_SHAPE, "sizes exceed the 32-bit row indices");
+  if (mode < GBW_MODE_AUTO || mode > GBW_MODE_GEMV)
+    return fail(GBW_ERR_SHAPE, "unknown mode");
+  if (!offsets || !w || !scale) return fail(GBW_ERR_NULL, "NULL weights or offsets");
+  if (P > 0 && (!x || !out)) return fail(GBW_ERR_NULL, "NULL x or out");
+  if (!row_to_token && T < P)
+    return fail(GBW_ERR_SHAPE, "row_to_token == NULL needs T >= P");
+  if (row_to_token && P > 0 && T < 1) return fail(GBW_ERR_SHAPE, "T must be >= 1");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out))
+    return fail(GBW_ERR_ALIGN, "x, packed weights and out must be 16-byte aligned");
+  if (f == Fmt::NF4 && !aligned4(scale)) return fail(GBW_ERR_ALIGN, "absmax must be 4-byte aligned");
+  if (!aligned4(offsets) || (row_to_token && !aligned4(row_to_token)))
+    return fail(GBW_ERR_ALIGN, "offsets / row_to_token must be 4-byte aligned");
+  if (mode == GBW_MODE_GEMM && K % 64)
+    return fail(GBW_ERR_SHAPE, "the tensor-core path needs K % 64 == 0");
+  int* err = nullptr;
+  int sms = 0;
+  gbw_status st = device_state(&err, &sms);
+  if (st != GBW_OK) return st;
+  if (P == 0) return GBW_OK;
+  GroupedProblem pb{x, T, K, w, scale, E, N, offsets, row_to_token, P, out, err};
+  const bool gemv = mode == GBW_MODE_GEMV || (mode == GBW_MODE_AUTO && (P <= 8 || K % 64));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = gemv ? launch_gemv(f, pb, sms, s) : launch_gemm(f, pb, sms, s);
+  return e == cudaSuccess ? GBW_OK : launch_error(e);
+}
+
+}  // namespace
+}  // namespace gbw
+
+using namespace gbw;
+
+extern "C" {
+
+gbw_status gnf4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
+                             const uint8_t* packed, const float* absmax,
+                             int32_t E, int64_t N,
+                             const int32_t* expert_offsets,
+                             const int32_t* row_to_token, int64_t P,
+                             uint16_t* out, int32_t mode, void* stream) {
+  return grouped_forward(Fmt::NF4, x, T, K, packed, absmax, E, N,
+                         expert_offsets, row_to_token, P, out, mode, stream);
+}
+
+gbw_status gmxfp4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
+                               const uint8_t* blocks, const uint8_t* scales,
+                               int32_t E, int64_t N,
+                               const int32_t* expert_offsets,
+                               const int32_t* row_to_token, int64_t P,
+                               uint16_t* out, int32_t mode, void* stream) {
+  return grouped_forward(Fmt::MXFP4, x, T, K, blocks, scales, E, N,
+                         expert_offsets, row_to_token, P, out, mode, stream);
+}
+
+gbw_status gnf4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
+                              const uint8_t* packed, const float* absmax,
+                              int32_t E, int64_t K,
+                              const int32_t* expert_offsets, uint16_t* dx,
+                              void* stream) {
+  if (P < 0 || N <= 0 || K <= 0 || E < 1)
+    return fail(GBW_ERR_SHAPE, "need P >= 0, N > 0, K > 0, E >= 1");
+  if (K % 64 || N % 64) return fail(GBW_ERR_SHAPE, "dgrad needs K % 64 == 0 and N % 64 == 0");
+  if (K > (int64_t)1 << 30 || P > INT32_MAX || (int64_t)E * N > INT32_MAX)
+    return fail(GBW_ERR_SHAPE, "sizes exceed the 32-bit row indices");
+  if (!packed || !absmax || !expert_offsets) return fail(GBW_ERR_NULL, "NULL weights or offsets");
+  if (P > 0 && (!dy || !dx)) return fail(GBW_ERR_NULL, "NULL dy or dx");
+  if (!aligned16(dy) || !aligned16(packed) || !aligned16(dx))
+    return fail(GBW_ERR_ALIGN, "dy, packed and dx must be 16-byte aligned");
+  if (!aligned4(absmax) || !aligned4(expert_offsets))
+    return fail(GBW_ERR_ALIGN, "absmax / offsets must be 4-byte aligned");
+  int* err = nullptr;
+  int sms = 0;
+  gbw_status st = device_state(&err, &sms);
+  if (st != GBW_OK) return st;
+  if (P == 0) return GBW_OK;
+  GroupedProblem pb{dy, P, K, packed, absmax, E, N, expert_offsets, nullptr, P, dx, err};
+  cudaError_t e = launch_dgrad(pb, sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GBW_OK : launch_error(e);
+}
+
+gbw_status gnf4_dequant(const uint8_t* packed, const float* absmax,
+                        int64_t rows, int64_t K, uint16_t* w_out,
+                        void* stream) {
+  if (rows < 0 || K <= 0 || K % 64) return fail(GBW_ERR_SHAPE, "need rows >= 0, K % 64 == 0");
+  if (rows > 0 && (!packed || !absmax || !w_out)) return fail(GBW_ERR_NULL, "NULL argument");
+  if (!aligned16(packed) || !aligned16(w_out) || !aligned4(absmax))
+    return fail(GBW_ERR_ALIGN, "packed / w_out must be 16-byte aligned");
+  int* err = nullptr;
+  int sms = 0;
+  gbw_status st = device_state(&err, &sms);
+  if (st != GBW_OK) return st;
+  cudaError_t e = launch_dequant(Fmt::NF4, packed, absmax, rows, K, w_out,
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GBW_OK : launch_error(e);
+}
+
+gbw_status gmxfp4_dequant(const uint8_t* blocks, const uint8_t* scales,
+                          int64_t rows, int64_t K, uint16_t* w_out,
+                          void* stream) {
+  if (rows < 0 || K <= 0 || K % 32) return fail(GBW_ERR_SHAPE, "need rows >= 0, K % 32 == 0");
+  if (rows > 0 && (!blocks || !scales || !w_out)) return fail(GBW_ERR_NULL, "NULL argument");
+  if (!aligned16(blocks) || !aligned16(w_out))
+    return fail(GBW_ERR_ALIGN, "blocks / w_out must be 16-byte aligned");
+  int* err = nullptr;
+  int sms = 0;
+  gbw_status st = device_state(&err, &sms);
+  if (st != GBW_OK) return st;
+  cudaError_t e = launch_dequant(Fmt::MXFP4, blocks, scales, rows, K, w_out,
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GBW_OK : launch_error(e);
+}
+
+gbw_status gnf4_quantize(const float* w, int64_t rows, int64_t K,
+                         uint8_t* packed, float* absmax, void* stream) {
+  if (rows < 0 || K <= 0 || K % 64) return fail(GBW_ERR_SHAPE, "need rows >= 0, K % 64 == 0");
+  if (rows > 0 && (!w || !packed || !absmax)) return fail(GBW_ERR_NULL, "NULL argument");
+  if (!aligned16(w) || !aligned4(absmax)) return fail(GBW_ERR_ALIGN, "w must be 16-byte aligned");
+  int* err = nullptr;
+  int sms = 0;
+  gbw_status st = device_state(&err, &sms);
+  if (st != GBW_OK) return st;
+  cudaError_t e = launch_quantize(Fmt::NF4, w, rows, K, packed, absmax,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GBW_OK : launch_error(e);
+}
+
+gbw_status gmxfp4_quantize(const float* w, int64_t rows, int64_t K,
+                           uint8_t* blocks, uint8_t* scales, void* stream) {
+  if (rows < 0 || K <= 0 || K % 32) return fail(GBW_ERR_SHAPE, "need rows >= 0, K % 32 == 0");
+  if (rows > 0 && (!w || !blocks || !scales)) return fail(GBW_ERR_NULL, "NULL argument");
+  if (!aligned16(w)) return fail(GBW_ERR_ALIGN, "w must be 16-byte aligned");
+  int* err = nullptr;
+  int sms = 0;
+  gbw_status st = device_state(&err, &sms);
+  if (st != GBW_OK) return st;
+  cudaError_t e = launch_quantize(Fmt::MXFP4, w, rows, K, blocks, scales,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GBW_OK : launch_error(e);
+}
+
+gbw_status gbw_device_status(void* stream, int32_t* host_err, int32_t clear) {
+  int* err = nullptr;
+  int sms = 0;
+  gbw_status st = device_state(&err, &sms);
+  if (st != GBW_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && clear && v) {
+    const int zero = 0;
+    e = cudaMemcpyAsync(err, &zero, sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) return launch_error(e);
+  if (host_err) *host_err = v;
+  return v ? GBW_ERR_DEVICE : GBW_OK;
+}
+
+const char* gbw_status_string(gbw_status s) {
+  switch (s) {
+    case GBW_OK: return "ok";
+    case GBW_ERR_NULL: return g_msg[0] ? g_msg : "NULL pointer";
+    case GBW_ERR_SHAPE: return g_msg[0] ? g_msg : "unsupported size";
+    case GBW_ERR_ALIGN: return g_msg[0] ? g_msg : "misaligned pointer";
+    case GBW_ERR_ARCH: return g_msg[0] ? g_msg : "device is not sm_100";
+    case GBW_ERR_LAUNCH: return g_msg[0] ? g_msg : "CUDA launch failed";
+    case GBW_ERR_DEVICE: return "device error word set (see GBW_DEVERR_* bits)";
+  }
+  return "unknown status";
+}
+
+int32_t gbw_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,382 @@
+// common.cuh -- device-side building blocks shared by the kernels of
+// libgbw: launch arguments, the device error word, bounded mbarrier waits,
+// TMA (cp.async.bulk.tensor) and tcgen05 (5th-generation tensor core /
+// tensor memory) wrappers for sm_100a.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gbw.h"
+
+namespace gbw {
+
+// ----------------------------------------------------------------------
+// launch arguments
+// ----------------------------------------------------------------------
+
+// One grouped projection: routed rows sorted by expert, E experts of weight
+// [N, K] in a 4-bit packed format.
+struct GroupedProblem {
+  const uint16_t* x;       // [T, K] bf16 (forward) or dy [P, N] (dgrad)
+  int64_t T;
+  int64_t K;
+  const uint8_t* w;        // packed codes [E, N, K/2]
+  const void* scale;       // NF4: float [E, N, K/64]; MXFP4: uint8 [E, N, K/32]
+  int32_t E;
+  int64_t N;
+  const int32_t* offsets;  // [E+1] device
+  const int32_t* row_to_token;  // [P] device or nullptr
+  int64_t P;
+  uint16_t* out;           // [P, N] bf16 (forward) or dx [P, K] (dgrad)
+  int* err;                // device error word
+};
+
+enum class Fmt : int { NF4 = 0, MXFP4 = 1 };
+
+// Host-side launchers (one per kernel family).  Each returns the CUDA
+// error of its launch.
+cudaError_t launch_dequant(Fmt f, const uint8_t* w, const void* scale,
+                           int64_t rows, int64_t K, uint16_t* out,
+                           cudaStream_t s);
+cudaError_t launch_quantize(Fmt f, const float* w, int64_t rows, int64_t K,
+                            uint8_t* codes, void* scale, cudaStream_t s);
+cudaError_t launch_gemv(Fmt f, const GroupedProblem& p, int num_sms,
+                        cudaStream_t s);
+cudaError_t launch_gemm(Fmt f, const GroupedProblem& p, int num_sms,
+                        cudaStream_t s);
+cudaError_t launch_dgrad(const GroupedProblem& p, int num_sms, cudaStream_t s);
+
+// ----------------------------------------------------------------------
+// device error word
+// ----------------------------------------------------------------------
+
+__device__ __forceinline__ void raise_error(int* err, int bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// ----------------------------------------------------------------------
+// small helpers
+// ----------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Two fp32 -> bf16x2, round to nearest even; `lo` lands in bits 15:0.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ----------------------------------------------------------------------
+// mbarrier (shared memory barriers with transaction counts)
+// ----------------------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar,
+                                                      uint32_t bytes) {
+  asm volatile(
+      "mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait budget of every pipeline wait: after this many nanoseconds without
+// progress the wait gives up, raises GBW_DEVERR_TIMEOUT and the kernel
+// unwinds instead of hanging the GPU.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Bounded wait for the phase with `parity` to complete.  `abort` is a
+// shared flag: once any thread of the CTA has given up, every other wait
+// returns false at once.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 63u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        raise_error(err, GBW_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait that ignores the abort flag, used while unwinding to let copies and
+// MMAs already in flight finish before shared or tensor memory is released.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// ----------------------------------------------------------------------
+// TMA (tensor memory accelerator)
+// ----------------------------------------------------------------------
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m))
+               : "memory");
+}
+
+// 2-D tiled load of box {c0.., c1..} into shared memory, completion counted
+// in bytes on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m,
+                                            int32_t c0, int32_t c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Row gather: four rows r0..r3 of a 2-D tensor, columns c0 .. c0+box-1,
+// written as four consecutive box rows at dst (swizzle of the map applies).
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m,
+                                            int32_t c0, int32_t r0, int32_t r1,
+                                            int32_t r2, int32_t r3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ----------------------------------------------------------------------
+// tcgen05: tensor memory and the 5th-generation MMA
+// ----------------------------------------------------------------------
+
+// Allocates `ncols` TMEM columns (power of two >= 32) for this CTA; the
+// base address is written to *dst_smem.  Whole warp.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile(
+      "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+          smem_u32(dst_smem)),
+      "r"(ncols)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile(
+      "tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
+      "r"(ncols)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Arrive on `bar` once every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
+      "[%0];" ::"r"(smem_u32(bar))
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (bf16 inputs, fp32 accum).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem,
+                                          uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16.
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc,
+                                          uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M x N tile.
+// a_mn / b_mn select the MN-major (transposed) smem layout.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(uint32_t M, uint32_t N,
+                                                       uint32_t a_mn,
+                                                       uint32_t b_mn) {
+  return (1u << 4)            // D format: f32
+         | (1u << 7)          // A format: bf16
+         | (1u << 10)         // B format: bf16
+         | (a_mn << 15)       // A major
+         | (b_mn << 16)       // B major
+         | ((N >> 3) << 17)   // N / 8
+         | ((M >> 4) << 24);  // M / 16
+}
+
+// Shared-memory matrix descriptor for a 128-byte-swizzled operand.
+//   lbo / sbo: leading / stride byte offsets (see the canonical layouts:
+//   K-major -> sbo = distance between 8-row groups; MN-major -> lbo =
+//   distance between 64-element atoms along MN, sbo = distance between
+//   8-row groups along K).
+__device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr,
+                                                     uint32_t lbo,
+                                                     uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;  // descriptor version for sm_100
+  d |= (uint64_t)2u << 61;  // layout: SWIZZLE_128B
+  return d;
+}
+
+// 32 lanes x 32 columns of 32-bit TMEM cells <-> 32 registers per thread:
+// thread t of the warp owns lane (warp's lane base + t).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr,
+                                                   const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, "
+      "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, "
+      "%22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+      "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
+      "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+      "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
+      "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr,
+                                                   uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, "
+      "%8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, "
+      "%22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+        "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]),
+        "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------
+// grouped-row bookkeeping
+// ----------------------------------------------------------------------
+
+// Loads expert_offsets into shared memory as a clamped running maximum in
+// [0, P] (so every row range stays inside the caller's buffers) and flags
+// any change the clamp made.  off_s has E+1 entries.  Whole block.
+__device__ __forceinline__ void load_offsets_clamped(const int32_t* offsets,
+                                                     int32_t E, int64_t P,
+                                                     int32_t* off_s, int* err) {
+  if (threadIdx.x == 0) {
+    int32_t prev = 0;
+    bool bad = false;
+    for (int32_t e = 0; e <= E; ++e) {
+      int32_t v = offsets[e];
+      int32_t c = v < prev ? prev : v;
+      if (c > (int32_t)P) c = (int32_t)P;
+      if (e == 0 && c != 0) c = 0;
+      if (e == E) c = (int32_t)P;
+      if (c != v) bad = true;
+      off_s[e] = c;
+      prev = c;
+    }
+    if (bad) raise_error(err, GBW_DEVERR_OFFSETS);
+  }
+  __syncthreads();
+}
+
+// Expert whose row range holds row p (binary search, p in [0, P)).
+__device__ __forceinline__ int32_t expert_of_row(const int32_t* off_s,
+                                                 int32_t E, int32_t p) {
+  int32_t lo = 0, hi = E - 1;
+  while (lo < hi) {
+    int32_t mid = (lo + hi + 1) >> 1;
+    if (off_s[mid] <= p) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int32_t token_of_row(const int32_t* r2t, int32_t p,
+                                                int64_t T, int* err) {
+  if (!r2t) return p;
+  int32_t t = __ldg(r2t + p);
+  if (t < 0 || t >= T) {
+    raise_error(err, GBW_DEVERR_TOKEN);
+    t = t < 0 ? 0 : (int32_t)(T - 1);
+  }
+  return t;
+}
+
+}  // namespace gbw

@@ -1,0 +1,311 @@
+// dgrad.cu -- grouped NF4 activation gradient dx = dy * W on tcgen05.
+//
+// "grouped-nf4-gemm 0.43.0", "Which entry point?": dgrad_4bit_grouped;
+// "Receipts-driven engineering": the NF4 path is differentiable and
+// fine-tuning never leaves the packed format.  For out = x W^T per expert,
+//   dx[p, k] = sum_n dy[p, n] * W_e(p)[n, k].
+// The reduction now runs over the weight rows n, and the absmax blocks lie
+// along the output dimension k, so the weights are read packed in the
+// transposed orientation.
+//
+// B200 design (one persistent CTA per SM, 16 warps):
+//   tile = 128 routed rows (MMA M) x 256 output columns k (MMA N), reduced
+//          over N in stages of 64 weight rows;
+//   warp 0      TMA: dy tile [128 x 64] (128B swizzle, K-major A operand)
+//               and the packed slab [64 weight rows x 128 bytes] (swizzled so
+//               the decode reads are bank-conflict free) -> smem ring (4)
+//   warps 4-11  decode: thread (weight row n, 64-wide k block j) decodes 64
+//               weights with the register table and stores them as one
+//               128-byte row of the MN-major, 128B-swizzled B operand
+//               (3-stage ring); the decoded tile lives only in smem
+//   warp 1      tcgen05.mma (A and B from smem, fp32 accumulator in TMEM)
+//   warps 12-15 epilogue: tcgen05.ld -> bf16 -> 16-byte stores of dx rows;
+//               two TMEM accumulators (2 x 256 columns) let the epilogue of
+//               one tile overlap the mainloop of the next.
+// Tiles (expert, k tile, routed-row tile) with routed-row tiles innermost, so
+// CTAs running together share one packed weight slab through L2.
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace gbw {
+namespace {
+
+constexpr int BM = 128;   // routed rows per tile (MMA M)
+constexpr int BN = 256;   // output k columns per tile (MMA N)
+constexpr int BR = 64;    // weight rows (reduction) per stage
+constexpr int LS = 4;     // load ring stages (dy + packed)
+constexpr int DS = 3;     // decoded-B ring stages
+constexpr int kThreads = 512;
+constexpr uint32_t kTmemCols = 512;
+
+constexpr int kAStageBytes = BM * BR * 2;   // 16 KB
+constexpr int kWStageBytes = BR * BN / 2;   // 8 KB
+constexpr int kLStageBytes = kAStageBytes + kWStageBytes;
+constexpr int kBStageBytes = BR * BN * 2;   // 32 KB
+
+struct Smem {
+  static constexpr int ld = 0;
+  static constexpr int b = ld + LS * kLStageBytes;
+  static constexpr int bars = b + DS * kBStageBytes;
+  static constexpr int nbars = 2 * LS + 2 * DS + 4 + 1;
+  static constexpr int misc = bars + nbars * 8;
+  static constexpr int tables = misc + 16;
+};
+
+struct DTile {
+  int32_t e, k0, p0, nv;
+};
+
+__device__ __forceinline__ DTile dtile_info(int64_t t, const int32_t* off,
+                                            const int32_t* ts, int32_t E) {
+  int32_t lo = 0, hi = E - 1;
+  while (lo < hi) {
+    int32_t mid = (lo + hi + 1) >> 1;
+    if (ts[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  const int32_t cnt = off[lo + 1] - off[lo];
+  const int32_t mt_n = (cnt + BM - 1) / BM;
+  const int32_t u = (int32_t)(t - ts[lo]);
+  const int32_t kt = u / mt_n, mt = u - kt * mt_n;
+  DTile d;
+  d.e = lo;
+  d.k0 = kt * BN;
+  d.p0 = off[lo] + mt * BM;
+  d.nv = min(BM, cnt - mt * BM);
+  return d;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
+             const __grid_constant__ CUtensorMap tmw) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::bars);
+  uint64_t* ld_full = bars;
+  uint64_t* ld_empty = ld_full + LS;
+  uint64_t* b_full = ld_empty + LS;
+  uint64_t* b_empty = b_full + DS;
+  uint64_t* acc_full = b_empty + DS;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
+  int32_t* off_s = reinterpret_cast<int32_t*>(smem + Smem::tables);
+  int32_t* ts_s = off_s + (pb.E + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t E = pb.E;
+  const int64_t N = pb.N;  // reduction length (weight rows)
+  const int64_t K = pb.K;  // output width
+  const int NS = (int)(N / BR);
+  const int32_t nkt = (int32_t)((K + BN - 1) / BN);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < LS; ++i) { mbar_init(&ld_full[i], 1); mbar_init(&ld_empty[i], 1 + 8); }
+    for (int i = 0; i < DS; ++i) { mbar_init(&b_full[i], 8); mbar_init(&b_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tma);
+    tma_prefetch_desc(&tmw);
+  }
+  load_offsets_clamped(pb.offsets, E, pb.P, off_s, pb.err);
+  if (threadIdx.x == 0) {
+    int32_t acc = 0;
+    for (int32_t e = 0; e < E; ++e) {
+      ts_s[e] = acc;
+      const int32_t cnt = off_s[e + 1] - off_s[e];
+      acc += nkt * ((cnt + BM - 1) / BM);
+    }
+    ts_s[E] = acc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t ntiles = ts_s[E];
+
+  if (warp == 0) {
+    // ---------------- loads: dy tile + packed slab ----------------
+    if (lane == 0) {
+      uint32_t g = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const DTile d = dtile_info(t, off_s, ts_s, E);
+        for (int ks = 0; ks < NS; ++ks, ++g) {
+          const uint32_t s = g % LS, ph = (g / LS) & 1u;
+          if (!(ok = mbar_wait(&ld_empty[s], ph ^ 1u, abort, pb.err))) break;
+          uint8_t* st = smem + Smem::ld + s * kLStageBytes;
+          mbar_arrive_expect_tx(&ld_full[s], kLStageBytes);
+          tma_load_2d(st, &tma, ks * BR, d.p0, &ld_full[s]);
+          tma_load_2d(st + kAStageBytes, &tmw, d.k0 / 2,
+                      (int32_t)((int64_t)d.e * N + (int64_t)ks * BR), &ld_full[s]);
+        }
+      }
+      if (*abort)
+        for (uint32_t i = (g > LS ? g - LS : 0); i < g; ++i)
+          mbar_drain(&ld_full[i % LS], (i / LS) & 1u);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t g = 0, it = 0;
+      bool ok = true;
+      const uint32_t ldbase = smem_u32(smem + Smem::ld);
+      const uint32_t bbase = smem_u32(smem + Smem::b);
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+        const DTile d = dtile_info(t, off_s, ts_s, E);
+        const uint32_t nmma = (uint32_t)min((int64_t)BN, K - d.k0);
+        const uint32_t idesc = make_idesc_bf16(BM, nmma, 0, 1);
+        const uint32_t ab = it & 1u;
+        if (!(ok = mbar_wait(&acc_empty[ab], ((it >> 1) & 1u) ^ 1u, abort, pb.err))) break;
+        tc_fence_after();
+        const uint32_t dacc = tmem + ab * 256u;
+        for (int ks = 0; ks < NS; ++ks, ++g) {
+          const uint32_t ls = g % LS, bs = g % DS;
+          if (!(ok = mbar_wait(&ld_full[ls], (g / LS) & 1u, abort, pb.err))) break;
+          if (!(ok = mbar_wait(&b_full[bs], (g / DS) & 1u, abort, pb.err))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < BR / 16; ++j) {
+            const uint64_t adesc =
+                make_sdesc_sw128(ldbase + ls * kLStageBytes + j * 32, 16, 1024);
+            const uint64_t bdesc =
+                make_sdesc_sw128(bbase + bs * kBStageBytes + j * 8192, 1024, 4096);
+            tc_mma_ss(dacc, adesc, bdesc, idesc, (ks | j) != 0);
+          }
+          tc_commit(&ld_empty[ls]);
+          tc_commit(&b_empty[bs]);
+        }
+        if (ok) tc_commit(&acc_full[ab]);
+      }
+      tc_commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ---------------- decode into the MN-major B operand ----------------
+    const int dw = warp - 4;
+    const int j = dw >> 1;                      // 64-wide k block of the tile
+    const int n = ((dw & 1) << 5) | lane;       // weight row within the stage
+    const int rr = n & 7;                       // row inside the 8-row atom
+    uint32_t g = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      const DTile d = dtile_info(t, off_s, ts_s, E);
+      const bool jvalid = d.k0 + 64 * j < K;
+      for (int ks = 0; ks < NS; ++ks, ++g) {
+        const uint32_t ls = g % LS, bs = g % DS;
+        const int64_t wrow = (int64_t)d.e * N + (int64_t)ks * BR + n;
+        float a = 0.0f;
+        if (jvalid)
+          a = __ldg(reinterpret_cast<const float*>(pb.scale) + wrow * (K / 64) +
+                    d.k0 / 64 + j);
+        ok = __all_sync(0xffffffffu, mbar_wait(&ld_full[ls], (g / LS) & 1u, abort, pb.err));
+        if (!ok) break;
+        // packed slab row n, bytes 32j .. 32j+31, stored 128B-swizzled
+        const uint8_t* wst = smem + Smem::ld + ls * kLStageBytes + kAStageBytes + n * 128;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(wst + (((2 * j) ^ rr) << 4));
+        const uint4 q1 = *reinterpret_cast<const uint4*>(wst + (((2 * j + 1) ^ rr) << 4));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ld_empty[ls]);
+        uint32_t o[32];
+        const uint32_t P[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        const Planes tb = nf4_planes(a);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) decode_word<true>(P[i], tb, &o[4 * i]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&b_empty[bs], ((g / DS) & 1u) ^ 1u, abort, pb.err));
+        if (!ok) break;
+        if (jvalid) {
+          // K-row n of atom (n/8, j): 128 bytes, chunk c at (c ^ rr)
+          uint8_t* dst = smem + Smem::b + bs * kBStageBytes + ((n >> 3) * 4 + j) * 1024 + rr * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(dst + ((c ^ rr) << 4)) =
+                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        }
+        // generic-proxy smem writes -> visible to the tensor core (async proxy)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b_full[bs]);
+      }
+    }
+  } else if (warp >= 12) {
+    // ---------------- epilogue ----------------
+    const uint32_t q = (uint32_t)warp & 3u;
+    const int m = (int)(q * 32 + lane);
+    uint32_t it = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      const DTile d = dtile_info(t, off_s, ts_s, E);
+      const uint32_t ab = it & 1u;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (it >> 1) & 1u, abort, pb.err));
+      if (!ok) break;
+      tc_fence_after();
+      const int width = (int)min((int64_t)BN, K - d.k0);
+      const int nchunks = width >> 5;
+      const uint32_t taddr = tmem + ((q * 32u) << 16) + ab * 256u;
+      uint16_t* dst = pb.out + (int64_t)(d.p0 + m) * K + d.k0;
+      for (int c = 0; c < nchunks; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, r);
+        tmem_wait_ld();
+        if (c == nchunks - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        }
+        if (m < d.nv) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+            o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+            o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+            o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+            reinterpret_cast<uint4*>(dst + c * 32)[v] = o;
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base,
+                        uint64_t d0, uint64_t d1, uint64_t pitch, uint32_t b0,
+                        uint32_t b1, CUtensorMapSwizzle sw);
+
+cudaError_t launch_dgrad(const GroupedProblem& pb, int num_sms, cudaStream_t s) {
+  if (pb.P == 0 || pb.K == 0) return cudaSuccess;
+  CUtensorMap tma, tmw;
+  // dy [P, N] bf16: box 64 (reduction) x 128 rows, 128B swizzle
+  cudaError_t e = make_map_2d(&tma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pb.x,
+                              (uint64_t)pb.N, (uint64_t)pb.P, (uint64_t)pb.N * 2,
+                              BR, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  // packed [E*N, K/2] u8: box 128 bytes x 64 rows, 128B swizzle
+  e = make_map_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.w, (uint64_t)pb.K / 2,
+                  (uint64_t)pb.E * (uint64_t)pb.N, (uint64_t)pb.K / 2, BN / 2, BR,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  const size_t smem = 1024 + Smem::tables + sizeof(int32_t) * 2 * (size_t)(pb.E + 1);
+  e = cudaFuncSetAttribute(dgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  dgrad_kernel<<<num_sms, kThreads, smem, s>>>(pb, tma, tmw);
+  return cudaGetLastError();
+}
+
+}  // namespace gbw

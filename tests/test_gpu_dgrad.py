@@ -1,0 +1,59 @@
+"""Grouped NF4 activation gradient against the CPU oracle."""
+import numpy as np
+import pytest
+
+import oracle as orc
+from grouped_bit_weight_b200 import synth
+from parity import assert_rows_close
+
+pytestmark = pytest.mark.gpu
+
+gbw = pytest.importorskip("grouped_bit_weight_b200")
+from gpu_util import bits, packed_weights, sample_rows, to_dev  # noqa: E402
+
+
+def _dgrad(dy, codes, scale, off):
+    import torch
+    dx = gbw.gnf4_grouped_dgrad(to_dev(dy), to_dev(codes), to_dev(scale), to_dev(off))
+    torch.cuda.synchronize()
+    assert gbw.device_status() == 0
+    return bits(dx)
+
+
+def test_tiny_dgrad():
+    off, _ = synth.tiny_routing(0)
+    codes, scale, wdec = packed_weights("nf4", 8, 256, 512, 1.0, 1)
+    P = int(off[-1])
+    dy = synth.to_bf16_bits(synth.normal((P, 256), 3, std=1e-2))
+    _, ref = orc.grouped_dgrad(dy, wdec, off, want_f64=True)
+    worst = assert_rows_close(_dgrad(dy, codes, scale, off), ref, what="tiny dgrad")
+    assert worst < 0.1
+
+
+def test_dgrad_ragged_edges():
+    """Empty experts, a 3-tile expert with a ragged tail, K = 320 (the last
+    output tile is 64 wide), N = 192."""
+    E, N, K = 4, 192, 320
+    counts = np.array([0, 300, 5, 0], np.int32)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    codes, scale, wdec = packed_weights("nf4", E, N, K, 1.0, 2)
+    dy = synth.to_bf16_bits(synth.normal((int(off[-1]), N), 4, std=1e-2))
+    _, ref = orc.grouped_dgrad(dy, wdec, off, want_f64=True)
+    assert_rows_close(_dgrad(dy, codes, scale, off), ref, what="ragged dgrad")
+
+
+@pytest.mark.parametrize("layer", [synth.QWEN_GATE_UP, synth.QWEN_DOWN])
+def test_dgrad_full_size(layer):
+    """Training dgrad on the Qwen3-30B-A3B prefill routing: dY [32768, N]
+    N(0, 1e-2); sampled rows checked."""
+    off, _ = synth.prefill_routing()
+    codes, scale, wdec = packed_weights("nf4", layer.E, layer.N, layer.K, layer.w_std, 21)
+    P = int(off[-1])
+    dy = synth.to_bf16_bits(synth.normal((P, layer.N), 22, std=1e-2))
+    got = _dgrad(dy, codes, scale, off)
+    rows = sample_rows(off, 32, 23)
+    sp = np.repeat(rows, layer.K)
+    sk = np.tile(np.arange(layer.K), len(rows))
+    ref = orc.grouped_dgrad_sampled(dy, wdec, off, sp, sk).reshape(len(rows), layer.K)
+    worst = assert_rows_close(got[rows], ref, what=f"{layer.name} dgrad")
+    assert worst < 0.1
