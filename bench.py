@@ -1,0 +1,612 @@
+"""Benchmark of the grouped 4-bit MoE matmul library on B200.
+
+Headline (one JSON line on rank 0): the Qwen3-30B-A3B-shaped NF4 decode
+layer -- one token routed to 8 of 128 experts, gate_up (N=1536, K=2048) then
+down (N=2048, K=768) through the bandwidth GEMV -- as HBM GB/s of
+algorithmic bytes (packed codes + scales of the active experts + x + out).
+A step is one such layer.  Consecutive steps rotate over 16 disjoint expert
+sets, so a step never finds its 21 MB of weights in the 126 MB L2 (340 MB are
+cycled).  Steps run as CUDA-graph replays.
+
+Also measured on one GPU and reported under "secondary": Qwen3 prefill
+(32768 routed rows) and the NF4 training dgrad on the tensor-core path,
+gpt-oss-20b MXFP4 at 2048 tokens (tensor cores) and at one token (GEMV).
+
+--impl reference times the CPU oracle (the plain fp64 definition) on the same
+decode workload on the host cores.
+Multi-GPU (torchrun): every rank runs an independent replica of the same
+workload (the layer has no exchange step); value = all ranks' bytes / the
+slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "grouped 4-bit MoE GEMM TFLOP/s (prefill) and decode GB/s, % of B200 roofline"
+WORKLOAD = ("qwen3_30b_a3b_nf4_decode: E=128, top-8, 1 token; gate_up N=1536 K=2048 "
+            "then down N=2048 K=768; weights N(0,0.02) NF4-packed, x N(0,1) bf16")
+N_SETS = 16  # disjoint 8-expert sets cycled by consecutive steps
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]),
+                float(p["bf16_tflops_sustained"]), "measured")
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- units
+
+def gemv_bytes(fmt, P, N, K, T_rows):
+    """Algorithmic bytes of one grouped GEMV launch: the active experts'
+    packed codes and scales (P rows, one per expert), x read once, out."""
+    codes = P * N * K // 2
+    scales = P * N * (K // 64) * 4 if fmt == "nf4" else P * N * (K // 32)
+    return codes + scales + T_rows * K * 2 + P * N * 2
+
+
+def gemm_flops(P, N, K):
+    return 2.0 * P * N * K
+
+
+# ---------------------------------------------------------------- clocks
+
+class Clocks:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.p = None
+        return self
+
+    def __exit__(self, *a):
+        self.rows = []
+        if self.p is None:
+            return
+        time.sleep(0.25)
+        self.p.terminate()
+        try:
+            out, _ = self.p.communicate(timeout=5)
+        except Exception:
+            self.p.kill()
+            out = ""
+        for line in out.strip().splitlines():
+            f = [s.strip() for s in line.split(",")]
+            if len(f) >= 8:
+                self.rows.append(f)
+
+    def summary(self):
+        rows = getattr(self, "rows", [])
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        pw = [num(r[2]) for r in rows if num(r[2]) is not None]
+        busy = [s for s, p in zip(sm, pw) if p is not None and p > 250] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v == "Active"})
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max((num(r[1]) or 0) for r in rows),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------- GPU side
+
+def make_nf4(torch, gbw, E, N, K, std, gen, dev):
+    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=dev)
+    scale = torch.empty((E, N, K // 64), dtype=torch.float32, device=dev)
+    for e in range(E):  # one expert at a time keeps the fp32 staging small
+        w = torch.randn((N, K), generator=gen, device=dev) * std
+        c, s = gbw.gnf4_quantize(w)
+        codes[e].copy_(c)
+        scale[e].copy_(s)
+    return codes, scale
+
+
+def make_mxfp4(torch, gbw, E, N, K, std, gen, dev):
+    codes = torch.empty((E, N, K // 32, 16), dtype=torch.uint8, device=dev)
+    scale = torch.empty((E, N, K // 32), dtype=torch.uint8, device=dev)
+    for e in range(E):
+        w = torch.randn((N, K), generator=gen, device=dev) * std
+        c, s = gbw.gmxfp4_quantize(w)
+        codes[e].copy_(c)
+        scale[e].copy_(s)
+    return codes, scale
+
+
+def event_time_ms(torch, fn, iters, stream):
+    """Average device time of fn() over iters calls, CUDA events on the
+    launching stream, synchronised on both sides."""
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def decode_routing(E, k, n_sets, seed):
+    """Disjoint expert sets; set j routes one token to experts perm[k*j:k*(j+1)]."""
+    from grouped_bit_weight_b200 import synth
+    perm = np.random.default_rng(seed).permutation(E)
+    return [synth.decode_routing(E, k, 0, experts=np.sort(perm[k * j:k * (j + 1)]))
+            for j in range(n_sets)]
+
+
+def run_ours(args, rank, world, dev):
+    import torch
+    import grouped_bit_weight_b200 as gbw
+    from grouped_bit_weight_b200 import synth
+
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + rank)
+    launches = {"n": 0}
+
+    # ---- the decode layer (headline) ----
+    GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
+    wgu = make_nf4(torch, gbw, GU.E, GU.N, GU.K, GU.w_std, gen, dev)
+    wdn = make_nf4(torch, gbw, DN.E, DN.N, DN.K, DN.w_std, gen, dev)
+    sets = decode_routing(GU.E, 8, N_SETS, seed=5)
+    offs = [torch.from_numpy(o).to(dev) for o, _ in sets]
+    r2ts = [torch.from_numpy(r).to(dev) for _, r in sets]
+    x_gu = (torch.randn((1, GU.K), generator=gen, device=dev)).to(torch.bfloat16)
+    x_dn = (torch.randn((8, DN.K), generator=gen, device=dev)).to(torch.bfloat16)
+    out_gu = torch.empty((8, GU.N), dtype=torch.bfloat16, device=dev)
+    out_dn = torch.empty((8, DN.N), dtype=torch.bfloat16, device=dev)
+
+    def step(j):
+        gbw.gnf4_grouped_gemm(x_gu, wgu[0], wgu[1], offs[j], r2ts[j], out=out_gu)
+        gbw.gnf4_grouped_gemm(x_dn, wdn[0], wdn[1], offs[j], None, out=out_dn)
+
+    bytes_gu = gemv_bytes("nf4", 8, GU.N, GU.K, 1)
+    bytes_dn = gemv_bytes("nf4", 8, DN.N, DN.K, 8)
+    bytes_step = bytes_gu + bytes_dn
+
+    for j in range(N_SETS):  # eager warm-up of every kernel / attribute
+        step(j)
+    torch.cuda.synchronize()
+    assert gbw.device_status(dev) == 0
+
+    graphs = []
+    for j in range(N_SETS):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(j)
+        graphs.append(g)
+    cycle = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(cycle):
+        for j in range(N_SETS):
+            step(j)
+
+    def run_steps(n):
+        for _ in range(n // N_SETS):
+            cycle.replay()
+        for j in range(n % N_SETS):
+            graphs[j].replay()
+
+    run_steps(args.warmup)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        run_steps(args.steps)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    launches["n"] += 2 * args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_per_step = ms / args.steps
+    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+
+    # dominant kernel: the gate_up GEMV alone, back to back in a graph of
+    # one launch per expert set; average device time per launch
+    gu_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gu_graph):
+        for j in range(N_SETS):
+            gbw.gnf4_grouped_gemm(x_gu, wgu[0], wgu[1], offs[j], r2ts[j], out=out_gu)
+    gu_ms = event_time_ms(torch, gu_graph.replay, 40, stream) / N_SETS
+    launches["n"] += 0  # the roofline loop runs outside the timed region
+    achieved = bytes_gu / (gu_ms * 1e-3) / 1e9
+    traffic = load_traffic("gemv_nf4_qwen3_decode_gate_up")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "traffic": traffic, "kernel": "gemv_kernel<NF4> (gate_up)",
+                "timing": "graph of 16 back-to-back launches, CUDA events, per-launch mean",
+                "algorithmic_bytes_per_launch": bytes_gu,
+                "launch_ms": round(gu_ms, 5), "peak_source": peak_kind}
+
+    # e2e: host buffers, copies inside the timed region, public API calls
+    e2e = measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step)
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "weights": "nf4 (absmax fp32 per 64)",
+                   "activations": "bf16", "experts_cycled": f"{N_SETS} disjoint sets of 8",
+                   "l2": "inputs larger than L2: 340 MB of packed weights cycled, 21 MB per step",
+                   "path": "bandwidth GEMV (GBW_MODE_AUTO picks it for P <= 8)",
+                   "graphs": "steps replayed as CUDA graphs",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": launches["n"],
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_secondary:
+        result["secondary"] = secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind)
+        result["gpu_launches"] = launches["n"]
+    return result
+
+
+def load_traffic(name):
+    """DRAM bytes per launch from the committed ncu summary, if present."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            return json.load(f).get(name)
+    except Exception:
+        return None
+
+
+def measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step):
+    """Same decode layer through the public API with host buffers: every step
+    copies its inputs (x, offsets, row map) from pinned host memory and
+    reads both outputs back; one synchronisation per step."""
+    from grouped_bit_weight_b200 import synth
+    GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
+    h_xgu = torch.randn((1, GU.K)).to(torch.bfloat16).pin_memory()
+    h_xdn = torch.randn((8, DN.K)).to(torch.bfloat16).pin_memory()
+    h_off = [torch.from_numpy(o).pin_memory() for o, _ in sets]
+    h_r2t = [torch.from_numpy(r).pin_memory() for _, r in sets]
+    h_ogu = torch.empty((8, GU.N), dtype=torch.bfloat16).pin_memory()
+    h_odn = torch.empty((8, DN.N), dtype=torch.bfloat16).pin_memory()
+    d_xgu = torch.empty_like(h_xgu, device=dev)
+    d_xdn = torch.empty_like(h_xdn, device=dev)
+    d_off = torch.empty_like(h_off[0], device=dev)
+    d_r2t = torch.empty_like(h_r2t[0], device=dev)
+    d_ogu = torch.empty((8, GU.N), dtype=torch.bfloat16, device=dev)
+    d_odn = torch.empty((8, DN.N), dtype=torch.bfloat16, device=dev)
+    bi = (h_xgu.numel() + h_xdn.numel()) * 2 + h_off[0].numel() * 4 + h_r2t[0].numel() * 4
+    bo = (h_ogu.numel() + h_odn.numel()) * 2
+
+    def one(j):
+        d_xgu.copy_(h_xgu, non_blocking=True)
+        d_xdn.copy_(h_xdn, non_blocking=True)
+        d_off.copy_(h_off[j], non_blocking=True)
+        d_r2t.copy_(h_r2t[j], non_blocking=True)
+        gbw.gnf4_grouped_gemm(d_xgu, wgu[0], wgu[1], d_off, d_r2t, out=d_ogu)
+        gbw.gnf4_grouped_gemm(d_xdn, wdn[0], wdn[1], d_off, None, out=d_odn)
+        h_ogu.copy_(d_ogu, non_blocking=True)
+        h_odn.copy_(d_odn, non_blocking=True)
+        stream.synchronize()
+
+    n = max(16, min(args.steps, 2000))
+    for j in range(32):
+        one(j % N_SETS)
+    torch.cuda.synchronize()
+    t = time.perf_counter()
+    for i in range(n):
+        one(i % N_SETS)
+    dt = time.perf_counter() - t
+    return {"value": round(bytes_step * n / dt / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": n,
+            "timing": "host wall clock around steps that each end in a stream sync"}
+
+
+def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):
+    out = []
+
+    def tc_entry(name, flops, fn, iters=20):
+        for _ in range(3):
+            fn()
+        ms = event_time_ms(torch, fn, iters, stream)
+        tf = flops / (ms * 1e-3) / 1e12
+        return {"workload": name, "value": round(tf, 1), "unit": "TFLOP/s",
+                "ms": round(ms, 4),
+                "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                             "peak": bf16, "unit": "TFLOP/s",
+                             "frac": round(tf / bf16, 4), "peak_source": peak_kind}}
+
+    # Qwen3-30B-A3B prefill, NF4, tensor cores
+    GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
+    off, r2t = synth.prefill_routing()
+    P = int(off[-1])
+    d_off = torch.from_numpy(off).to(dev)
+    d_r2t = torch.from_numpy(r2t).to(dev)
+    wgu = make_nf4(torch, gbw, GU.E, GU.N, GU.K, GU.w_std, gen, dev)
+    x = torch.randn((4096, GU.K), generator=gen, device=dev).to(torch.bfloat16)
+    o = torch.empty((P, GU.N), dtype=torch.bfloat16, device=dev)
+    out.append(tc_entry("qwen3 prefill gate_up NF4 (P=32768, N=1536, K=2048)",
+                        gemm_flops(P, GU.N, GU.K),
+                        lambda: gbw.gnf4_grouped_gemm(x, wgu[0], wgu[1], d_off, d_r2t, out=o)))
+    dy = (torch.randn((P, GU.N), generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
+    dx = torch.empty((P, GU.K), dtype=torch.bfloat16, device=dev)
+    out.append(tc_entry("qwen3 dgrad gate_up NF4 (P=32768, N=1536, K=2048)",
+                        gemm_flops(P, GU.N, GU.K),
+                        lambda: gbw.gnf4_grouped_dgrad(dy, wgu[0], wgu[1], d_off, out=dx)))
+    del wgu, x, o, dy, dx
+    wdn = make_nf4(torch, gbw, DN.E, DN.N, DN.K, DN.w_std, gen, dev)
+    xd = torch.randn((P, DN.K), generator=gen, device=dev).to(torch.bfloat16)
+    od = torch.empty((P, DN.N), dtype=torch.bfloat16, device=dev)
+    out.append(tc_entry("qwen3 prefill down NF4 (P=32768, N=2048, K=768)",
+                        gemm_flops(P, DN.N, DN.K),
+                        lambda: gbw.gnf4_grouped_gemm(xd, wdn[0], wdn[1], d_off, None, out=od)))
+    dyd = (torch.randn((P, DN.N), generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
+    dxd = torch.empty((P, DN.K), dtype=torch.bfloat16, device=dev)
+    out.append(tc_entry("qwen3 dgrad down NF4 (P=32768, N=2048, K=768)",
+                        gemm_flops(P, DN.N, DN.K),
+                        lambda: gbw.gnf4_grouped_dgrad(dyd, wdn[0], wdn[1], d_off, out=dxd)))
+    del wdn, xd, od, dyd, dxd
+    torch.cuda.empty_cache()
+
+    # gpt-oss-20b MXFP4: 2048 tokens (tensor cores) and 1 token (GEMV)
+    for L in (synth.GPTOSS_GATE_UP, synth.GPTOSS_DOWN):
+        w = make_mxfp4(torch, gbw, L.E, L.N, L.K, L.w_std, gen, dev)
+        off, r2t = synth.uniform_routing(2048, L.E, 4, seed=7)
+        P = int(off[-1])
+        d_off, d_r2t = torch.from_numpy(off).to(dev), torch.from_numpy(r2t).to(dev)
+        x = torch.randn((2048, L.K), generator=gen, device=dev).to(torch.bfloat16)
+        o = torch.empty((P, L.N), dtype=torch.bfloat16, device=dev)
+        out.append(tc_entry(f"gpt-oss-20b {L.name.split('_')[-1]} MXFP4 batch 2048 (P=8192, N={L.N}, K={L.K})",
+                            gemm_flops(P, L.N, L.K),
+                            lambda: gbw.gmxfp4_grouped_gemm(x, w[0], w[1], d_off, d_r2t, out=o)))
+        sets = decode_routing(L.E, 4, 8, seed=9)
+        offs = [torch.from_numpy(a).to(dev) for a, _ in sets]
+        r2ts = [torch.from_numpy(b).to(dev) for _, b in sets]
+        x1 = torch.randn((1, L.K), generator=gen, device=dev).to(torch.bfloat16)
+        o1 = torch.empty((4, L.N), dtype=torch.bfloat16, device=dev)
+        for j in range(8):
+            gbw.gmxfp4_grouped_gemm(x1, w[0], w[1], offs[j], r2ts[j], out=o1)
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1):
+            for j in range(8):
+                gbw.gmxfp4_grouped_gemm(x1, w[0], w[1], offs[j], r2ts[j], out=o1)
+        ms = event_time_ms(torch, g1.replay, 40, stream) / 8
+        nbytes = gemv_bytes("mxfp4", 4, L.N, L.K, 1)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.append({"workload": f"gpt-oss-20b {L.name.split('_')[-1]} MXFP4 batch 1 (P=4, N={L.N}, K={L.K}), 8 expert sets cycled",
+                    "value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 5),
+                    "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                                 "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                                 "peak_source": peak_kind}})
+        del w, x, o
+        torch.cuda.empty_cache()
+    torch.cuda.synchronize()
+    assert gbw.device_status(dev) == 0
+    return out
+
+
+# ---------------------------------------------------------------- single cases
+
+def run_case(args, dev):
+    """One kernel on one workload, `--warmup` then `--steps` launches, for
+    profiling (ncu -k / -s / -c pick launches out of this command)."""
+    import torch
+    import grouped_bit_weight_b200 as gbw
+    from grouped_bit_weight_b200 import synth
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(99)
+    c = args.case
+    if c in ("decode_gate_up", "decode_down"):
+        L = synth.QWEN_GATE_UP if c == "decode_gate_up" else synth.QWEN_DOWN
+        w = make_nf4(torch, gbw, L.E, L.N, L.K, L.w_std, gen, dev)
+        sets = decode_routing(L.E, 8, N_SETS, seed=5)
+        offs = [torch.from_numpy(o).to(dev) for o, _ in sets]
+        r2ts = [torch.from_numpy(r).to(dev) for _, r in sets]
+        T = 1 if L is synth.QWEN_GATE_UP else 8
+        x = torch.randn((T, L.K), generator=gen, device=dev).to(torch.bfloat16)
+        o = torch.empty((8, L.N), dtype=torch.bfloat16, device=dev)
+        it = {"i": 0}
+        def fn():
+            j = it["i"] % N_SETS
+            it["i"] += 1
+            gbw.gnf4_grouped_gemm(x, w[0], w[1], offs[j], r2ts[j] if T == 1 else None, out=o)
+        nbytes, unit = gemv_bytes("nf4", 8, L.N, L.K, T), "GB/s"
+    elif c in ("prefill_gate_up", "prefill_down", "dgrad_gate_up", "dgrad_down"):
+        L = synth.QWEN_GATE_UP if c.endswith("gate_up") else synth.QWEN_DOWN
+        off, r2t = synth.prefill_routing()
+        P = int(off[-1])
+        d_off, d_r2t = torch.from_numpy(off).to(dev), torch.from_numpy(r2t).to(dev)
+        w = make_nf4(torch, gbw, L.E, L.N, L.K, L.w_std, gen, dev)
+        if c.startswith("prefill"):
+            T = 4096 if L is synth.QWEN_GATE_UP else P
+            x = torch.randn((T, L.K), generator=gen, device=dev).to(torch.bfloat16)
+            o = torch.empty((P, L.N), dtype=torch.bfloat16, device=dev)
+            rt = d_r2t if T == 4096 else None
+            fn = lambda: gbw.gnf4_grouped_gemm(x, w[0], w[1], d_off, rt, out=o)
+        else:
+            dy = (torch.randn((P, L.N), generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
+            o = torch.empty((P, L.K), dtype=torch.bfloat16, device=dev)
+            fn = lambda: gbw.gnf4_grouped_dgrad(dy, w[0], w[1], d_off, out=o)
+        nbytes, unit = gemm_flops(P, L.N, L.K), "TFLOP/s"
+    elif c in ("mxfp4_2048_gate_up", "mxfp4_2048_down", "mxfp4_1_gate_up", "mxfp4_1_down"):
+        L = synth.GPTOSS_GATE_UP if c.endswith("gate_up") else synth.GPTOSS_DOWN
+        w = make_mxfp4(torch, gbw, L.E, L.N, L.K, L.w_std, gen, dev)
+        T = 2048 if "_2048_" in c else 1
+        off, r2t = (synth.uniform_routing(T, L.E, 4, seed=7) if T > 1
+                    else synth.decode_routing(L.E, 4, 0))
+        P = int(off[-1])
+        d_off, d_r2t = torch.from_numpy(off).to(dev), torch.from_numpy(r2t).to(dev)
+        x = torch.randn((T, L.K), generator=gen, device=dev).to(torch.bfloat16)
+        o = torch.empty((P, L.N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: gbw.gmxfp4_grouped_gemm(x, w[0], w[1], d_off, d_r2t, out=o)
+        nbytes, unit = ((gemm_flops(P, L.N, L.K), "TFLOP/s") if T > 1
+                        else (gemv_bytes("mxfp4", P, L.N, L.K, 1), "GB/s"))
+    else:
+        raise SystemExit(f"unknown case {c}")
+    for _ in range(args.warmup):
+        fn()
+    ms = event_time_ms(torch, fn, args.steps, stream)
+    assert gbw.device_status(dev) == 0
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    print(json.dumps({"case": c, "ms": round(ms, 5), "launches": args.steps,
+                      "value": round(nbytes / (ms * 1e-3) / scale, 2), "unit": unit}))
+
+
+# ---------------------------------------------------------------- oracle side
+
+def oracle_decode_step_fn():
+    """One decode layer by the CPU oracle: decode the 8 active experts'
+    weights, then the fp64 grouped matmuls (inputs drawn on the CPU)."""
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import oracle as orc
+    from grouped_bit_weight_b200 import synth
+    GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
+    pg = orc.nf4_pack(synth.normal((8, GU.N, GU.K), 31, GU.w_std))
+    pd = orc.nf4_pack(synth.normal((8, DN.N, DN.K), 32, DN.w_std))
+    xg = synth.to_bf16_bits(synth.normal((1, GU.K), 33))
+    xd = synth.to_bf16_bits(synth.normal((8, DN.K), 34))
+    off = np.arange(9, dtype=np.int32)        # one row per active expert
+    r2t = np.zeros(8, np.int32)
+
+    def step():
+        wg = orc.nf4_decode(pg[0], pg[1], GU.K, bf16=True)
+        orc.grouped_forward(xg, wg, off, r2t)
+        wd = orc.nf4_decode(pd[0], pd[1], DN.K, bf16=True)
+        orc.grouped_forward(xd, wd, off, None)
+    return step, orc.num_threads()
+
+
+def run_reference(args):
+    from grouped_bit_weight_b200 import synth
+    GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
+    step, cores = oracle_decode_step_fn()
+    nbytes = gemv_bytes("nf4", 8, GU.N, GU.K, 1) + gemv_bytes("nf4", 8, DN.N, DN.K, 8)
+    for _ in range(max(1, min(args.warmup, 3))):
+        step()
+    n = max(1, min(args.steps, 40))
+    t = time.perf_counter()
+    for _ in range(n):
+        step()
+    dt = time.perf_counter() - t
+    v = nbytes * n / dt / 1e9
+    sample = f"{n} full decode layers (8 experts x gate_up + down), fp64 oracle"
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+            "n_gpus": 1, "steps": n, "warmup": args.warmup,
+            "ms_per_step": round(dt / n * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "runs_on": "host CPU cores"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def cpu_baseline():
+    """The oracle, as it stands, on ~10-30 s of the decode workload."""
+    from grouped_bit_weight_b200 import synth
+    GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
+    step, cores = oracle_decode_step_fn()
+    nbytes = gemv_bytes("nf4", 8, GU.N, GU.K, 1) + gemv_bytes("nf4", 8, DN.N, DN.K, 8)
+    step()
+    n, t = 0, time.perf_counter()
+    while time.perf_counter() - t < 10.0 and n < 200:
+        step()
+        n += 1
+    dt = time.perf_counter() - t
+    return {"value": round(nbytes * n / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{n} full decode layers (8 experts, gate_up + down) in {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=3200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="time one kernel on one workload (profiling helper)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    dev = torch.device("cuda", local)
+    if args.case:
+        run_case(args, dev)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    res = run_ours(args, rank, world, dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -353,10 +353,11 @@ int orc_grouped_forward(const uint16_t* x, int64_t T, int64_t K,
   }
   for (int32_t e = 0; e < E; ++e) {
     const uint16_t* W = wdec + (int64_t)e * N * K;
-#pragma omp parallel for schedule(static)
-    for (int64_t p = off[e]; p < off[e + 1]; ++p) {
-      const uint16_t* xr = x + (row_to_token ? (int64_t)row_to_token[p] : p) * K;
+    const int64_t p0 = off[e], p1 = off[e + 1];
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t p = p0; p < p1; ++p) {
       for (int64_t n = 0; n < N; ++n) {
+        const uint16_t* xr = x + (row_to_token ? (int64_t)row_to_token[p] : p) * K;
         const uint16_t* wr = W + n * K;
         double s = 0.0;
         for (int64_t k = 0; k < K; ++k)

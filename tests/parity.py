@@ -44,3 +44,20 @@ def assert_rows_close(gpu_bf16_bits, oracle_f64, rel: float = 1e-2, what=""):
     ok, worst, n = check_rows(gpu_bf16_bits, oracle_f64, rel)
     assert ok, f"{what}: {n} elements, worst |err|/tol = {worst:.3g} (> 1)"
     return worst
+
+
+def assert_rows_exact_operands(gpu_bf16_bits, oracle_f64, rel_acc=1e-4, what=""):
+    """Stricter check for paths whose bf16 operands equal the oracle's decoded
+    weights exactly: the only differences left are fp32 accumulation order
+    (bounded here by rel_acc * rms(row)) and the final rounding to bf16
+    (half an ulp of the value).  A weight decoded even 2^-9 off would move
+    outputs by ~1e-3 * rms and fail."""
+    g = bf16_bits_to_f64(gpu_bf16_bits)
+    o = np.asarray(oracle_f64, np.float64)
+    assert g.shape == o.shape and o.size > 0
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True))
+    bound = 0.5 * np.maximum(bf16_ulp(o), bf16_ulp(g)) + rel_acc * rms
+    err = np.abs(g - o)
+    ratio = float(np.max(err / bound))
+    assert np.all(err <= bound), f"{what}: worst |err|/bound = {ratio:.3g}"
+    return ratio

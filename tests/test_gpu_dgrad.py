@@ -4,7 +4,7 @@ import pytest
 
 import oracle as orc
 from grouped_bit_weight_b200 import synth
-from parity import assert_rows_close
+from parity import assert_rows_close, assert_rows_exact_operands
 
 pytestmark = pytest.mark.gpu
 
@@ -26,8 +26,9 @@ def test_tiny_dgrad():
     P = int(off[-1])
     dy = synth.to_bf16_bits(synth.normal((P, 256), 3, std=1e-2))
     _, ref = orc.grouped_dgrad(dy, wdec, off, want_f64=True)
-    worst = assert_rows_close(_dgrad(dy, codes, scale, off), ref, what="tiny dgrad")
-    assert worst < 0.1
+    got = _dgrad(dy, codes, scale, off)
+    assert_rows_close(got, ref, what="tiny dgrad")
+    assert_rows_exact_operands(got, ref, what="tiny dgrad")
 
 
 def test_dgrad_ragged_edges():
@@ -39,7 +40,9 @@ def test_dgrad_ragged_edges():
     codes, scale, wdec = packed_weights("nf4", E, N, K, 1.0, 2)
     dy = synth.to_bf16_bits(synth.normal((int(off[-1]), N), 4, std=1e-2))
     _, ref = orc.grouped_dgrad(dy, wdec, off, want_f64=True)
-    assert_rows_close(_dgrad(dy, codes, scale, off), ref, what="ragged dgrad")
+    got = _dgrad(dy, codes, scale, off)
+    assert_rows_close(got, ref, what="ragged dgrad")
+    assert_rows_exact_operands(got, ref, what="ragged dgrad")
 
 
 @pytest.mark.parametrize("layer", [synth.QWEN_GATE_UP, synth.QWEN_DOWN])
@@ -55,5 +58,5 @@ def test_dgrad_full_size(layer):
     sp = np.repeat(rows, layer.K)
     sk = np.tile(np.arange(layer.K), len(rows))
     ref = orc.grouped_dgrad_sampled(dy, wdec, off, sp, sk).reshape(len(rows), layer.K)
-    worst = assert_rows_close(got[rows], ref, what=f"{layer.name} dgrad")
-    assert worst < 0.1
+    assert_rows_close(got[rows], ref, what=f"{layer.name} dgrad")
+    assert_rows_exact_operands(got[rows], ref, what=f"{layer.name} dgrad")
