@@ -194,6 +194,28 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m,
       : "memory");
 }
 
+// 16-byte asynchronous global -> shared copy (L2 only), grouped with
+// commit_group and waited for with wait_group.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+// Orders this thread's view of generic-proxy shared-memory writes before its
+// later async-proxy accesses (tensor core operand reads).
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation MMA
 // ----------------------------------------------------------------------
@@ -291,12 +313,18 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr,
 
 // 32 lanes x 32 columns of 32-bit TMEM cells <-> 32 registers per thread:
 // thread t of the warp owns lane (warp's lane base + t).
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr,
-                                                   const uint32_t (&r)[32]) {
+// tcgen05.st reads its source registers and tcgen05.ld writes its
+// destination registers asynchronously: the registers belong to the
+// operation until tcgen05.wait::st / wait::ld.  The wait therefore sits in
+// the same asm statement, so the compiler cannot reuse or read those
+// registers in between.
+__device__ __forceinline__ void tmem_store_32x32b_x32(uint32_t taddr,
+                                                      const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, "
       "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, "
-      "%22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "%22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
       "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
       "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
@@ -305,16 +333,14 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr,
       "r"(r[30]), "r"(r[31])
       : "memory");
 }
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
 
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr,
-                                                   uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_load_32x32b_x32(uint32_t taddr,
+                                                     uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, "
       "%8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, "
-      "%22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      "%22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
         "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]),
         "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
@@ -325,9 +351,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr,
       : "r"(taddr)
       : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 // ----------------------------------------------------------------------
 // grouped-row bookkeeping
@@ -335,26 +358,63 @@ __device__ __forceinline__ void tmem_wait_ld() {
 
 // Loads expert_offsets into shared memory as a clamped running maximum in
 // [0, P] (so every row range stays inside the caller's buffers) and flags
-// any change the clamp made.  off_s has E+1 entries.  Whole block.
+// any change the clamp made.  off_s has E+1 entries.  Whole block; valid
+// offsets (the normal case) are checked in parallel, only invalid ones take
+// the serial clamp.
 __device__ __forceinline__ void load_offsets_clamped(const int32_t* offsets,
                                                      int32_t E, int64_t P,
                                                      int32_t* off_s, int* err) {
-  if (threadIdx.x == 0) {
-    int32_t prev = 0;
-    bool bad = false;
-    for (int32_t e = 0; e <= E; ++e) {
-      int32_t v = offsets[e];
-      int32_t c = v < prev ? prev : v;
-      if (c > (int32_t)P) c = (int32_t)P;
-      if (e == 0 && c != 0) c = 0;
-      if (e == E) c = (int32_t)P;
-      if (c != v) bad = true;
-      off_s[e] = c;
-      prev = c;
-    }
-    if (bad) raise_error(err, GBW_DEVERR_OFFSETS);
+  int bad = 0;
+  for (int32_t e = threadIdx.x; e <= E; e += blockDim.x) {
+    const int32_t v = __ldg(offsets + e);
+    off_s[e] = v;
+    if (v < 0 || v > (int32_t)P || (e == 0 && v != 0) || (e == E && v != (int32_t)P))
+      bad = 1;
+    if (e < E && __ldg(offsets + e + 1) < v) bad = 1;
   }
-  __syncthreads();
+  if (__syncthreads_or(bad)) {
+    if (threadIdx.x == 0) {
+      int32_t prev = 0;
+      for (int32_t e = 0; e <= E; ++e) {
+        int32_t c = off_s[e] < prev ? prev : off_s[e];
+        if (c > (int32_t)P) c = (int32_t)P;
+        if (e == 0) c = 0;
+        if (e == E) c = (int32_t)P;
+        off_s[e] = c;
+        prev = c;
+      }
+      raise_error(err, GBW_DEVERR_OFFSETS);
+    }
+    __syncthreads();
+  }
+}
+
+// ts[e] = sum over experts e' < e of tiles(e'), ts[E] = total, where
+// tiles(e) = per_tile_n * ceil(count(e) / rows_per_tile).  Warp 0 scans 32
+// experts at a time with shuffles; the block must sync afterwards.
+__device__ __forceinline__ void tile_prefix(const int32_t* off_s, int32_t E,
+                                            int32_t rows_per_tile,
+                                            int32_t per_tile_n, int32_t* ts) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  int32_t carry = 0;
+  for (int32_t base = 0; base < E; base += 32) {
+    const int32_t e = base + lane;
+    int32_t v = 0;
+    if (e < E) {
+      const int32_t cnt = off_s[e + 1] - off_s[e];
+      v = per_tile_n * ((cnt + rows_per_tile - 1) / rows_per_tile);
+    }
+    int32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (e < E) ts[e] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) ts[E] = carry;
 }
 
 // Expert whose row range holds row p (binary search, p in [0, P)).

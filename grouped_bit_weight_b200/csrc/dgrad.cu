@@ -118,15 +118,7 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
     tma_prefetch_desc(&tmw);
   }
   load_offsets_clamped(pb.offsets, E, pb.P, off_s, pb.err);
-  if (threadIdx.x == 0) {
-    int32_t acc = 0;
-    for (int32_t e = 0; e < E; ++e) {
-      ts_s[e] = acc;
-      const int32_t cnt = off_s[e + 1] - off_s[e];
-      acc += nkt * ((cnt + BM - 1) / BM);
-    }
-    ts_s[E] = acc;
-  }
+  tile_prefix(off_s, E, BM, nkt, ts_s);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -196,46 +188,64 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
     const int j = dw >> 1;                      // 64-wide k block of the tile
     const int n = ((dw & 1) << 5) | lane;       // weight row within the stage
     const int rr = n & 7;                       // row inside the 8-row atom
-    uint32_t g = 0;
-    bool ok = true;
-    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      const DTile d = dtile_info(t, off_s, ts_s, E);
-      const bool jvalid = d.k0 + 64 * j < K;
-      for (int ks = 0; ks < NS; ++ks, ++g) {
-        const uint32_t ls = g % LS, bs = g % DS;
-        const int64_t wrow = (int64_t)d.e * N + (int64_t)ks * BR + n;
-        float a = 0.0f;
-        if (jvalid)
-          a = __ldg(reinterpret_cast<const float*>(pb.scale) + wrow * (K / 64) +
-                    d.k0 / 64 + j);
-        ok = __all_sync(0xffffffffu, mbar_wait(&ld_full[ls], (g / LS) & 1u, abort, pb.err));
-        if (!ok) break;
-        // packed slab row n, bytes 32j .. 32j+31, stored 128B-swizzled
-        const uint8_t* wst = smem + Smem::ld + ls * kLStageBytes + kAStageBytes + n * 128;
-        const uint4 q0 = *reinterpret_cast<const uint4*>(wst + (((2 * j) ^ rr) << 4));
-        const uint4 q1 = *reinterpret_cast<const uint4*>(wst + (((2 * j + 1) ^ rr) << 4));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ld_empty[ls]);
-        uint32_t o[32];
-        const uint32_t P[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        const Planes tb = nf4_planes(a);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) decode_word<true>(P[i], tb, &o[4 * i]);
-        ok = __all_sync(0xffffffffu, mbar_wait(&b_empty[bs], ((g / DS) & 1u) ^ 1u, abort, pb.err));
-        if (!ok) break;
-        if (jvalid) {
-          // K-row n of atom (n/8, j): 128 bytes, chunk c at (c ^ rr)
-          uint8_t* dst = smem + Smem::b + bs * kBStageBytes + ((n >> 3) * 4 + j) * 1024 + rr * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(dst + ((c ^ rr) << 4)) =
-                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        }
-        // generic-proxy smem writes -> visible to the tensor core (async proxy)
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b_full[bs]);
+    const int64_t my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const uint32_t total = (uint32_t)(my_tiles * NS);
+    // absmax of stage g for (row n, block j), fetched three stages ahead
+    int64_t pf_tile = -1;
+    int32_t pf_e = 0, pf_k0 = 0;
+    auto scale_at = [&](uint32_t g) -> float {
+      if (g >= total) return 0.0f;
+      const int64_t ti_idx = g / NS;
+      if (ti_idx != pf_tile) {
+        pf_tile = ti_idx;
+        const DTile d = dtile_info(blockIdx.x + ti_idx * gridDim.x, off_s, ts_s, E);
+        pf_e = d.e;
+        pf_k0 = d.k0;
       }
+      if (pf_k0 + 64 * j >= K) return 0.0f;
+      const int64_t wrow = (int64_t)pf_e * N + (int64_t)(g % NS) * BR + n;
+      return __ldg(reinterpret_cast<const float*>(pb.scale) + wrow * (K / 64) + pf_k0 / 64 + j);
+    };
+    float s0 = scale_at(0), s1 = scale_at(1), s2 = scale_at(2);
+    int64_t cur_tile = -1;
+    bool jvalid = false;
+    for (uint32_t g = 0; g < total; ++g) {
+      const float a = s0;
+      s0 = s1;
+      s1 = s2;
+      s2 = scale_at(g + 3);
+      const int64_t ti_idx = g / NS;
+      if (ti_idx != cur_tile) {
+        cur_tile = ti_idx;
+        const DTile d = dtile_info(blockIdx.x + ti_idx * gridDim.x, off_s, ts_s, E);
+        jvalid = d.k0 + 64 * j < K;
+      }
+      const uint32_t ls = g % LS, bs = g % DS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[ls], (g / LS) & 1u, abort, pb.err))) break;
+      // packed slab row n, bytes 32j .. 32j+31, stored 128B-swizzled
+      const uint8_t* wst = smem + Smem::ld + ls * kLStageBytes + kAStageBytes + n * 128;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(wst + (((2 * j) ^ rr) << 4));
+      const uint4 q1 = *reinterpret_cast<const uint4*>(wst + (((2 * j + 1) ^ rr) << 4));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ld_empty[ls]);
+      uint32_t o[32];
+      const uint32_t P[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const Planes tb = nf4_planes(a);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) decode_word<true>(P[i], tb, &o[4 * i]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&b_empty[bs], ((g / DS) & 1u) ^ 1u, abort, pb.err))) break;
+      if (jvalid) {
+        // K-row n of atom (n/8, j): 128 bytes, chunk c at (c ^ rr)
+        uint8_t* dst = smem + Smem::b + bs * kBStageBytes + ((n >> 3) * 4 + j) * 1024 + rr * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(dst + ((c ^ rr) << 4)) =
+              make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+      }
+      // generic-proxy smem writes -> visible to the tensor core (async proxy)
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b_full[bs]);
     }
   } else if (warp >= 12) {
     // ---------------- epilogue ----------------
@@ -254,8 +264,7 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
       uint16_t* dst = pb.out + (int64_t)(d.p0 + m) * K + d.k0;
       for (int c = 0; c < nchunks; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, r);
-        tmem_wait_ld();
+        tmem_load_32x32b_x32(taddr + c * 32, r);
         if (c == nchunks - 1) {
           tc_fence_before();
           __syncwarp();

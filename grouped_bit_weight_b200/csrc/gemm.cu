@@ -10,21 +10,29 @@
 //   tile  = 128 weight rows (MMA M) x up to 256 routed rows (MMA N) x K,
 //           i.e. the matmul runs as out^T = W x^T ("swap AB"), so an expert
 //           with few routed rows gets a narrow MMA N instead of a padded M;
-//   warp 0      TMA: packed weight tiles [128 rows x 32 B] -> smem ring (8)
-//   warp 2      TMA tile::gather4: the tile's x rows (through row_to_token)
-//               -> 128B-swizzled smem ring (4 stages of 64 K)
+//   warps 2-3   the tile's x rows -> 128B-swizzled smem ring (4 stages of
+//               64 K): one 2-D TMA tile per stage when routed row p reads x
+//               row p; 16-byte cp.async from 64 threads when rows are
+//               gathered through row_to_token (one TMA tile::gather4 per four
+//               rows measured ~4x slower: the TMA front end serialises them)
 //   warps 4-11  decode: each thread owns one weight row; per 64-K stage it
-//               reads its 32 packed bytes, builds the block's bf16 table and
-//               decodes with byte permutes, then writes 64 bf16 straight into
-//               tensor memory (tcgen05.st) as the MMA's A operand -- the
-//               decoded weights never touch shared or global memory; two
-//               groups of four warps take alternate stages
-//   warp 1      one thread issues tcgen05.mma (A from TMEM, B from smem,
-//               fp32 accumulator in TMEM) and tcgen05.commit
+//               loads its 32 packed bytes (one 32-byte sector) and the block
+//               scale straight from global memory, two of its stages ahead,
+//               builds the block's bf16 table and decodes with byte
+//               permutes, then stores the 64 bf16 as one
+//               128-byte row of the 128B-swizzled A tile (4-stage smem ring);
+//               two groups of four warps take alternate stages
+//   warp 1      one thread issues tcgen05.mma (A and B from smem, fp32
+//               accumulator in TMEM) and tcgen05.commit
 //   warps 12-15 epilogue: tcgen05.ld the 128 x N accumulator, round to bf16,
 //               transpose through smem, 16-byte stores of out rows
-// Tensor memory: columns [0,256) accumulator, [256,512) an 8-stage ring of
-// decoded A tiles (128 lanes x 32 columns of bf16x2 each).
+// Tensor memory holds two 128 x 256 fp32 accumulators, so the epilogue of
+// one tile overlaps the mainloop of the next.
+// (Staging the packed weights through a TMA ring of 128 x 32-byte boxes was
+// tried first: the decode warps on the three sub-partitions without the
+// issuing warp occasionally read bytes that differed from global memory
+// after the ring's full barrier had completed.  Per-thread sector loads
+// avoid the ring and measured exact.)
 // Scheduler: tiles (expert, 128-row weight tile, 256-row token tile) with
 // zero-row experts skipped, enumerated from expert_offsets by every CTA and
 // dealt round-robin (token tiles innermost, so CTAs running at the same time
@@ -39,24 +47,22 @@ constexpr int BM = 128;   // weight rows per tile (MMA M)
 constexpr int BT = 256;   // routed rows per tile (max MMA N)
 constexpr int BK = 64;    // K per stage
 constexpr int XS = 4;     // activation ring stages
-constexpr int WS = 8;     // packed-weight ring stages == TMEM A ring stages
+constexpr int AS = 4;     // decoded-weight (A operand) ring stages
 constexpr int kThreads = 512;
-constexpr uint32_t kAccCols = 256;
-constexpr uint32_t kACol0 = 256;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 
 constexpr int kXStageBytes = BT * BK * 2;      // 32 KB
-constexpr int kWStageBytes = BM * BK / 2;      // 4 KB
+constexpr int kAStageBytes = BM * BK * 2;      // 16 KB
 constexpr int kEpiRowBytes = 80;               // 64 B of data + 16 B pad
 constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
 
 struct Smem {
   // byte offsets inside the dynamic shared memory block
   static constexpr int x = 0;
-  static constexpr int w = x + XS * kXStageBytes;
-  static constexpr int epi = w + WS * kWStageBytes;
+  static constexpr int a = x + XS * kXStageBytes;
+  static constexpr int epi = a + AS * kAStageBytes;
   static constexpr int bars = epi + 4 * kEpiWarpBytes;
-  static constexpr int nbars = 2 * XS + 4 * WS + 3;
+  static constexpr int nbars = 2 * XS + 2 * AS + 5;
   static constexpr int misc = bars + nbars * 8;  // tmem base, abort flag
   static constexpr int tables = misc + 16;       // offsets[E+1], tile_start[E+1]
 };
@@ -88,8 +94,7 @@ __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
 
 template <Fmt F>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
-            const __grid_constant__ CUtensorMap tmw) {
+gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128B-swizzled activation tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -97,13 +102,11 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::bars);
   uint64_t* x_full = bars;
   uint64_t* x_empty = x_full + XS;
-  uint64_t* w_full = x_empty + XS;
-  uint64_t* w_empty = w_full + WS;
-  uint64_t* a_full = w_empty + WS;
-  uint64_t* a_empty = a_full + WS;
-  uint64_t* acc_full = a_empty + WS;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* mma_done = acc_empty + 1;
+  uint64_t* a_full = x_empty + XS;
+  uint64_t* a_empty = a_full + AS;
+  uint64_t* acc_full = a_empty + AS;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
   int32_t* off_s = reinterpret_cast<int32_t*>(smem + Smem::tables);
@@ -116,15 +119,16 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
   const int32_t ntn = (int32_t)((N + BM - 1) / BM);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < XS; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
-    for (int i = 0; i < WS; ++i) {
-      mbar_init(&w_full[i], 1);
-      mbar_init(&w_empty[i], 4);
+    const uint32_t xcount = pb.row_to_token ? 64u : 1u;  // 64 copy threads or one TMA
+    for (int i = 0; i < XS; ++i) { mbar_init(&x_full[i], xcount); mbar_init(&x_empty[i], 1); }
+    for (int i = 0; i < AS; ++i) {
       mbar_init(&a_full[i], 4);
       mbar_init(&a_empty[i], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
     mbar_init(mma_done, 1);
     *abort = 0;
     fence_barrier_init();
@@ -133,117 +137,112 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmx);
-    tma_prefetch_desc(&tmw);
-  }
+  if (warp == 2 && lane == 0) tma_prefetch_desc(&tmx);
   load_offsets_clamped(pb.offsets, E, pb.P, off_s, pb.err);  // has __syncthreads
-  if (threadIdx.x == 0) {
-    int32_t acc = 0;
-    for (int32_t e = 0; e < E; ++e) {
-      ts_s[e] = acc;
-      const int32_t cnt = off_s[e + 1] - off_s[e];
-      acc += ntn * ((cnt + BT - 1) / BT);
-    }
-    ts_s[E] = acc;
-  }
+  tile_prefix(off_s, E, BT, ntn, ts_s);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t ntiles = ts_s[E];
 
-  if (warp == 0) {
-    // ---------------- packed-weight producer ----------------
-    if (lane == 0) {
-      uint32_t g = 0;
-      bool ok = true;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
-        const int32_t row0 = (int32_t)((int64_t)ti.e * N + ti.n0);
-        for (int kb = 0; kb < NK; ++kb, ++g) {
-          const uint32_t s = g % WS, ph = (g / WS) & 1u;
-          if (!(ok = mbar_wait(&w_empty[s], ph ^ 1u, abort, pb.err))) break;
-          mbar_arrive_expect_tx(&w_full[s], kWStageBytes);
-          tma_load_2d(smem + Smem::w + s * kWStageBytes, &tmw, kb * (BK / 2), row0,
-                      &w_full[s]);
-        }
-      }
-      // after an abort, let the copies already issued land first
-      if (*abort)
-        for (uint32_t i = (g > WS ? g - WS : 0); i < g; ++i)
-          mbar_drain(&w_full[i % WS], (i / WS) & 1u);
-    }
-  } else if (warp == 2) {
-    // ---------------- activation producer (row gather) ----------------
+  if (warp == 2 || warp == 3) {
+    // ---------------- activation producer ----------------
     uint32_t g = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
-      const int ngroups = (ti.nv + 3) >> 2;  // gather4 groups (<= 64)
-      int32_t tok[2][4];
+    if (pb.row_to_token == nullptr) {
+      // routed row p reads x row p: one 2-D TMA tile (64 K x 256 rows) per stage
+      if (warp == 2 && lane == 0) {
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+          const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
+          for (int kb = 0; kb < NK; ++kb, ++g) {
+            const uint32_t s = g % XS, ph = (g / XS) & 1u;
+            if (!(ok = mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err))) break;
+            mbar_arrive_expect_tx(&x_full[s], kXStageBytes);
+            tma_load_2d(smem + Smem::x + s * kXStageBytes, &tmx, kb * BK, ti.p0, &x_full[s]);
+          }
+        }
+        if (*abort)
+          for (uint32_t i = (g > XS ? g - XS : 0); i < g; ++i)
+            mbar_drain(&x_full[i % XS], (i / XS) & 1u);
+      }
+    } else {
+      // gathered rows: 64 threads copy 16-byte chunks with cp.async, placing
+      // chunk c of row r at (c ^ (r % 8)) -- the 128-byte swizzle the MMA's
+      // descriptor expects.  cp.async writes through the generic proxy, so a
+      // thread publishes stage g only after its own copies of g have landed
+      // (wait_group) and a proxy fence; XS - 1 stages stay in flight.
+      constexpr int kLag = XS - 1;  // < XS, or the producer would wait on itself
+      const int pt = (warp - 2) * 32 + lane;  // rows pt, pt+64, pt+128, pt+192
+      uint32_t pub = 0;                       // stages published so far
+      auto publish_upto = [&](uint32_t upto) {
+        for (; pub < upto; ++pub) mbar_arrive(&x_full[pub % XS]);
+      };
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
+        const uint16_t* src[4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int gi = lane + 32 * h;
+        for (int i = 0; i < 4; ++i) {
+          const int r = pt + 64 * i;
+          src[i] = r < ti.nv
+                       ? pb.x + (int64_t)token_of_row(pb.row_to_token, ti.p0 + r, pb.T, pb.err) * K
+                       : nullptr;
+        }
+        for (int kb = 0; kb < NK; ++kb, ++g) {
+          const uint32_t s = g % XS, ph = (g / XS) & 1u;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err)))) break;
+          const uint32_t dst = smem_u32(smem + Smem::x + s * kXStageBytes);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          int32_t row = 4 * gi + r;
-          row = row < ti.nv ? row : ti.nv - 1;  // pad with the last valid row
-          tok[h][r] = gi < ngroups
-                          ? token_of_row(pb.row_to_token, ti.p0 + row, pb.T, pb.err)
-                          : 0;
+          for (int i = 0; i < 4; ++i) {
+            if (!src[i]) continue;
+            const int r = pt + 64 * i;
+            const uint16_t* sp = src[i] + kb * BK;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              cp_async_16(dst + r * 128 + ((c ^ (r & 7)) << 4), sp + c * 8);
+          }
+          cp_async_commit();
+          if (g + 1 > (uint32_t)kLag) {
+            cp_async_wait_group<kLag>();  // stage g - kLag has landed
+            fence_proxy_async();
+            publish_upto(g + 1 - kLag);
+          }
         }
       }
-      for (int kb = 0; kb < NK; ++kb, ++g) {
-        const uint32_t s = g % XS, ph = (g / XS) & 1u;
-        int good = 1;
-        if (lane == 0) {
-          good = mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err);
-          if (good) mbar_arrive_expect_tx(&x_full[s], (uint32_t)ngroups * 512u);
-        }
-        good = __shfl_sync(0xffffffffu, good, 0);
-        if (!good) { ok = false; break; }
-        uint8_t* dst = smem + Smem::x + s * kXStageBytes;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int gi = lane + 32 * h;
-          if (gi < ngroups)
-            tma_gather4(dst + gi * 512, &tmx, kb * BK, tok[h][0], tok[h][1],
-                        tok[h][2], tok[h][3], &x_full[s]);
-        }
-      }
+      cp_async_wait_all();
+      fence_proxy_async();
+      if (ok) publish_upto(g);
     }
-    if (lane == 0 && *abort)
-      for (uint32_t i = (g > XS ? g - XS : 0); i < g; ++i)
-        mbar_drain(&x_full[i % XS], (i / XS) & 1u);
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       uint32_t g = 0, it = 0;
       bool ok = true;
       const uint32_t xbase = smem_u32(smem + Smem::x);
+      const uint32_t abase = smem_u32(smem + Smem::a);
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
         const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
         const uint32_t nmma = (uint32_t)((ti.nv + 15) & ~15);
         const uint32_t idesc = make_idesc_bf16(BM, nmma, 0, 0);
-        if (!(ok = mbar_wait(acc_empty, (it & 1u) ^ 1u, abort, pb.err))) break;
+        const uint32_t ab = it & 1u;
+        if (!(ok = mbar_wait(&acc_empty[ab], ((it >> 1) & 1u) ^ 1u, abort, pb.err))) break;
         tc_fence_after();
+        const uint32_t dacc = tmem + ab * 256u;
         for (int kb = 0; kb < NK; ++kb, ++g) {
-          const uint32_t xs = g % XS, ws = g % WS;
-          if (!(ok = mbar_wait(&a_full[ws], (g / WS) & 1u, abort, pb.err))) break;
+          const uint32_t xs = g % XS, as = g % AS;
+          if (!(ok = mbar_wait(&a_full[as], (g / AS) & 1u, abort, pb.err))) break;
           if (!(ok = mbar_wait(&x_full[xs], (g / XS) & 1u, abort, pb.err))) break;
           tc_fence_after();
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t bdesc =
-                make_sdesc_sw128(xbase + xs * kXStageBytes + j * 32, 16, 1024);
-            tc_mma_ts(tmem, tmem + kACol0 + ws * 32 + j * 8, bdesc, idesc,
-                      (kb | j) != 0);
+            const uint64_t adesc = make_sdesc_sw128(abase + as * kAStageBytes + j * 32, 16, 1024);
+            const uint64_t bdesc = make_sdesc_sw128(xbase + xs * kXStageBytes + j * 32, 16, 1024);
+            tc_mma_ss(dacc, adesc, bdesc, idesc, (kb | j) != 0);
           }
           tc_commit(&x_empty[xs]);
-          tc_commit(&a_empty[ws]);
+          tc_commit(&a_empty[as]);
         }
-        if (ok) tc_commit(acc_full);
+        if (ok) tc_commit(&acc_full[ab]);
       }
       // every MMA this thread issued has finished before TMEM is released
       tc_commit(mma_done);
@@ -251,80 +250,96 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     }
   } else if (warp >= 4 && warp < 12) {
     // ---------------- decode ----------------
-    const uint32_t grp = (uint32_t)(warp - 4) >> 2;  // stage parity handled
-    const uint32_t q = (uint32_t)warp & 3u;          // TMEM lane quarter
+    const uint32_t grp = (uint32_t)(warp - 4) >> 2;  // takes stages g with g % 2 == grp
+    const uint32_t q = (uint32_t)warp & 3u;
     const int m = (int)(q * 32 + lane);              // weight row in tile
-    const uint32_t tlane = tmem + ((q * 32u) << 16);
-    uint32_t g = 0;
-    bool ok = true;
-    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
-      const bool rvalid = ti.n0 + m < N;
-      const int64_t wrow = (int64_t)ti.e * N + ti.n0 + m;
-      for (int kb = 0; kb < NK; ++kb, ++g) {
-        if ((g & 1u) != grp) continue;
-        const uint32_t ws = g % WS, ph = (g / WS) & 1u;
-        // block scale(s) of this row and stage
-        float a = 0.0f;
-        uint32_t s01 = 0;
-        if (rvalid) {
-          if (F == Fmt::NF4)
-            a = __ldg(reinterpret_cast<const float*>(pb.scale) + wrow * (K / 64) + kb);
-          else
-            s01 = __ldg(reinterpret_cast<const uint16_t*>(
-                reinterpret_cast<const uint8_t*>(pb.scale) + wrow * (K / 32) + 2 * kb));
-        }
-        ok = __all_sync(0xffffffffu, mbar_wait(&w_full[ws], ph, abort, pb.err));
-        if (!ok) break;
-        const uint4* src = reinterpret_cast<const uint4*>(smem + Smem::w + ws * kWStageBytes + m * 32);
-        const uint4 q0 = src[0], q1 = src[1];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&w_empty[ws]);
-        const uint32_t P[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        uint32_t o[32];
-        if (F == Fmt::NF4) {
-          const Planes tb = nf4_planes(a);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) decode_word<true>(P[i], tb, &o[4 * i]);
-        } else {
-          const Planes t0 = mxfp4_planes(s01 & 0xFFu);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) decode_word<false>(P[i], t0, &o[4 * i]);
-          const Planes t1 = mxfp4_planes(s01 >> 8);
-#pragma unroll
-          for (int i = 4; i < 8; ++i) decode_word<false>(P[i], t1, &o[4 * i]);
-        }
-        ok = __all_sync(0xffffffffu, mbar_wait(&a_empty[ws], ph ^ 1u, abort, pb.err));
-        if (!ok) break;
-        tc_fence_after();
-        tmem_st_32x32b_x32(tlane + kACol0 + ws * 32, o);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[ws]);
+    const int mr = m & 7;                            // row inside its 8-row atom
+    const int64_t my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const uint32_t total = (uint32_t)(my_tiles * NK);
+    // The row's 32 packed bytes and its block scale for stage g are read
+    // from global memory four stages (two of this group's) ahead of their
+    // use, so their latency overlaps decode work.
+    struct Pf { uint4 q0, q1; uint32_t sc; };
+    int64_t pf_tile = -1, pf_wrow = 0;
+    bool pf_valid = false;
+    auto fetch = [&](uint32_t g) -> Pf {
+      Pf f;
+      f.q0 = f.q1 = make_uint4(0u, 0u, 0u, 0u);
+      f.sc = 0u;
+      if (g >= total) return f;
+      const int64_t ti_idx = g / NK;
+      if (ti_idx != pf_tile) {
+        pf_tile = ti_idx;
+        const TileInfo ti = tile_info(blockIdx.x + ti_idx * gridDim.x, off_s, ts_s, E, ntn);
+        pf_valid = ti.n0 + m < N;
+        pf_wrow = (int64_t)ti.e * N + ti.n0 + m;
       }
+      if (!pf_valid) return f;
+      const int kb = (int)(g % NK);
+      const uint4* wp = reinterpret_cast<const uint4*>(pb.w + pf_wrow * (K / 2) + kb * (BK / 2));
+      f.q0 = __ldg(wp);
+      f.q1 = __ldg(wp + 1);
+      if (F == Fmt::NF4)
+        f.sc = __float_as_uint(__ldg(reinterpret_cast<const float*>(pb.scale) + pf_wrow * (K / 64) + kb));
+      else
+        f.sc = __ldg(reinterpret_cast<const uint16_t*>(
+            reinterpret_cast<const uint8_t*>(pb.scale) + pf_wrow * (K / 32) + 2 * kb));
+      return f;
+    };
+    Pf f0 = fetch(grp), f1 = fetch(grp + 2);
+    for (uint32_t g = grp; g < total; g += 2) {
+      const Pf cur = f0;
+      f0 = f1;
+      f1 = fetch(g + 4);
+      const uint32_t sv = cur.sc;
+      const uint32_t as = g % AS, aph = (g / AS) & 1u;
+      const uint32_t P[8] = {cur.q0.x, cur.q0.y, cur.q0.z, cur.q0.w,
+                             cur.q1.x, cur.q1.y, cur.q1.z, cur.q1.w};
+      uint32_t o[32];
+      if (F == Fmt::NF4) {
+        const Planes tb = nf4_planes(__uint_as_float(sv));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) decode_word<true>(P[i], tb, &o[4 * i]);
+      } else {
+        const Planes t0 = mxfp4_planes(sv & 0xFFu);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) decode_word<false>(P[i], t0, &o[4 * i]);
+        const Planes t1 = mxfp4_planes((sv >> 8) & 0xFFu);
+#pragma unroll
+        for (int i = 4; i < 8; ++i) decode_word<false>(P[i], t1, &o[4 * i]);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], aph ^ 1u, abort, pb.err))) break;
+      // row m of the K-major, 128B-swizzled A tile: chunk c at (c ^ (m % 8))
+      uint8_t* dst = smem + Smem::a + as * kAStageBytes + m * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(dst + ((c ^ mr) << 4)) =
+            make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+      fence_proxy_async();  // generic-proxy stores -> tensor core reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[as]);
     }
   } else if (warp >= 12) {
     // ---------------- epilogue ----------------
     const uint32_t q = (uint32_t)warp & 3u;
-    const uint32_t tlane = tmem + ((q * 32u) << 16);
     uint8_t* stage = smem + Smem::epi + q * kEpiWarpBytes;
     uint32_t it = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, it & 1u, abort, pb.err));
+      const uint32_t ab = it & 1u;
+      const uint32_t tlane = tmem + ((q * 32u) << 16) + ab * 256u;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (it >> 1) & 1u, abort, pb.err));
       if (!ok) break;
       tc_fence_after();
       const int nchunks = (ti.nv + 31) >> 5;
       const int ncol0 = ti.n0 + (int)q * 32;  // first output column of this warp
       for (int c = 0; c < nchunks; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tlane + c * 32, r);
-        tmem_wait_ld();
+        tmem_load_32x32b_x32(tlane + c * 32, r);
         if (c == nchunks - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
         // thread = output column ncol0+lane, r[j] = routed row c*32+j
 #pragma unroll
@@ -400,21 +415,19 @@ size_t gemm_smem_bytes(int32_t E) {
 cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
                         cudaStream_t s) {
   if (pb.P == 0 || pb.N == 0) return cudaSuccess;
-  CUtensorMap tmx, tmw;
+  CUtensorMap tmx;
+  // identity rows: tiles of 64 K x 256 rows; gathered rows use cp.async and
+  // never read this map
   cudaError_t e = make_map_2d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pb.x,
-                              (uint64_t)pb.K, (uint64_t)pb.T, (uint64_t)pb.K * 2,
-                              BK, 1, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (e != cudaSuccess) return e;
-  e = make_map_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.w, (uint64_t)pb.K / 2,
-                  (uint64_t)pb.E * (uint64_t)pb.N, (uint64_t)pb.K / 2, BK / 2, BM,
-                  CU_TENSOR_MAP_SWIZZLE_NONE);
+                              (uint64_t)pb.K, (uint64_t)(pb.T > 0 ? pb.T : 1),
+                              (uint64_t)pb.K * 2, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const size_t smem = gemm_smem_bytes(pb.E);
   auto k = (f == Fmt::NF4) ? gemm_kernel<Fmt::NF4> : gemm_kernel<Fmt::MXFP4>;
   e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<num_sms, kThreads, smem, s>>>(pb, tmx, tmw);
+  k<<<num_sms, kThreads, smem, s>>>(pb, tmx);
   return cudaGetLastError();
 }
 

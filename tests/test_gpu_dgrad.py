@@ -60,3 +60,27 @@ def test_dgrad_full_size(layer):
     ref = orc.grouped_dgrad_sampled(dy, wdec, off, sp, sk).reshape(len(rows), layer.K)
     assert_rows_close(got[rows], ref, what=f"{layer.name} dgrad")
     assert_rows_exact_operands(got[rows], ref, what=f"{layer.name} dgrad")
+
+
+def test_dgrad_repeatable():
+    """Repeated dgrad launches give identical bits (no pipeline races)."""
+    import torch
+    L = synth.QWEN_GATE_UP
+    off, _ = synth.prefill_routing()
+    P = int(off[-1])
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(41)
+    codes = torch.empty((L.E, L.N, L.K // 2), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((L.E, L.N, L.K // 64), dtype=torch.float32, device="cuda")
+    for e in range(L.E):
+        c, s = gbw.gnf4_quantize(torch.randn((L.N, L.K), generator=gen, device="cuda") * L.w_std)
+        codes[e].copy_(c)
+        sc[e].copy_(s)
+    dy = (torch.randn((P, L.N), generator=gen, device="cuda") * 1e-2).to(torch.bfloat16)
+    d_off = to_dev(off)
+    ref = gbw.gnf4_grouped_dgrad(dy, codes, sc, d_off)
+    for _ in range(4):
+        got = gbw.gnf4_grouped_dgrad(dy, codes, sc, d_off)
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    assert gbw.device_status() == 0

@@ -187,3 +187,50 @@ def test_corrupted_nibble_is_detected(mode):
     ok, worst, n = check_rows(got, ref)
     assert n > 0 and not ok, worst
     assert check_rows(_run("nf4", x, codes, scale, off, r2t, mode), ref)[0]
+
+
+def _device_layer(fmt, L, seed):
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    if fmt == "mxfp4":
+        codes = torch.empty((L.E, L.N, L.K // 32, 16), dtype=torch.uint8, device="cuda")
+        sc = torch.empty((L.E, L.N, L.K // 32), dtype=torch.uint8, device="cuda")
+        for e in range(L.E):
+            c, s = gbw.gmxfp4_quantize(torch.randn((L.N, L.K), generator=gen, device="cuda") * L.w_std)
+            codes[e].copy_(c)
+            sc[e].copy_(s)
+    else:
+        codes = torch.empty((L.E, L.N, L.K // 2), dtype=torch.uint8, device="cuda")
+        sc = torch.empty((L.E, L.N, L.K // 64), dtype=torch.float32, device="cuda")
+        for e in range(L.E):
+            c, s = gbw.gnf4_quantize(torch.randn((L.N, L.K), generator=gen, device="cuda") * L.w_std)
+            codes[e].copy_(c)
+            sc[e].copy_(s)
+    return codes, sc, gen
+
+
+@pytest.mark.parametrize("fmt,layer,tokens", [("mxfp4", synth.GPTOSS_GATE_UP, 2048),
+                                               ("mxfp4", synth.GPTOSS_DOWN, 2048),
+                                               ("nf4", synth.QWEN_GATE_UP, 4096)])
+def test_repeatable_and_path_independent(fmt, layer, tokens):
+    """The tensor-core path is deterministic: repeated launches give the same
+    bits, and gathering rows through row_to_token gives exactly the bits of
+    running on the pre-gathered rows (same decode, same MMA order).  A race
+    in the pipeline shows up here long before it exceeds the tolerance."""
+    if tokens == 4096:
+        off, r2t = synth.prefill_routing()
+    else:
+        off, r2t = synth.uniform_routing(tokens, layer.E, 4, seed=7)
+    codes, sc, gen = _device_layer(fmt, layer, 31)
+    x = torch.randn((tokens, layer.K), generator=gen, device="cuda").to(torch.bfloat16)
+    d_off, d_r2t = to_dev(off), to_dev(r2t)
+    xg = x[d_r2t.long()].contiguous()
+    fn = FWD[fmt]
+    ref = fn(xg, codes, sc, d_off, None, mode="gemm")
+    for _ in range(3):
+        a = fn(x, codes, sc, d_off, d_r2t, mode="gemm")
+        b = fn(xg, codes, sc, d_off, None, mode="gemm")
+        torch.cuda.synchronize()
+        assert torch.equal(a.view(torch.int16), ref.view(torch.int16))
+        assert torch.equal(b.view(torch.int16), ref.view(torch.int16))
+    assert gbw.device_status() == 0
