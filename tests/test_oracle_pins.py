@@ -340,3 +340,49 @@ def test_parity_check_has_teeth():
     assert n > 0 and not ok, worst
     with pytest.raises(AssertionError):
         check_rows(np.zeros((0, 4), np.uint16), np.zeros((0, 4)))
+
+
+# ------------------------------------------------------ golden fixtures
+
+def test_page_examples_fixture():
+    """The packers' printed worked examples (tests/golden/page_examples.json:
+    'grouped-nf4-gemm 0.43.0', 'Try the packers and byte checks on CPU',
+    examples 1 and 2): shapes, dtypes, the rounded relative error and the
+    byte-identical re-pack, on this repository's own N(0,1) draws."""
+    from golden_cases import load
+    g = load("page_examples.json")
+    n = g["nf4"]
+    w = synth.normal(tuple(n["w_shape"]), seed=0)
+    p, a = orc.nf4_pack(w)
+    assert list(p.shape) == n["packed_shape"] and p.dtype == np.dtype(n["packed_dtype"])
+    assert list(a.shape) == n["absmax_shape"] and a.dtype == np.dtype(n["absmax_dtype"])
+    wq = orc.nf4_decode(p, a, n["w_shape"][1])
+    rel = np.linalg.norm(wq - w) / np.linalg.norm(w)
+    assert round(float(rel), n["rel_err_digits"]) == n["rel_err_printed"], rel
+    assert np.array_equal(orc.nf4_pack(wq)[0], p) == n["repack_identical"]
+    m = g["mxfp4"]
+    w = synth.normal(tuple(m["w_shape"]), seed=0)
+    b, s = orc.mxfp4_pack(w)
+    assert list(b.shape) == m["blocks_shape"] and b.dtype == np.dtype(m["blocks_dtype"])
+    assert list(s.shape) == m["scales_shape"] and s.dtype == np.dtype(m["scales_dtype"])
+    wq = orc.mxfp4_decode(b, s)
+    rel = np.linalg.norm(wq - w) / np.linalg.norm(w)
+    assert round(float(rel), m["rel_err_digits"]) == m["rel_err_printed"], rel
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
+def test_hand_worked_grouped_matmul(fmt):
+    """tests/golden/hand_worked.json: bytes, scales, activations and routing
+    chosen so every product and sum is exact, with the outputs derived by
+    hand.  A flipped nibble order, a wrong sign bit, a scale off by one
+    power of two or a routing slip changes at least one of them."""
+    from golden_cases import hand_case
+    c = hand_case(fmt)
+    if fmt == "nf4":
+        wd = orc.nf4_decode(c["codes"], c["scale"], c["K"], bf16=True)
+    else:
+        wd = orc.mxfp4_decode(c["codes"], c["scale"], bf16=True)
+    x = orc.f32_to_bf16(c["x"])
+    out, o64 = orc.grouped_forward(x, wd, c["offsets"], c["row_to_token"], want_f64=True)
+    assert np.array_equal(o64, c["out"])
+    assert np.array_equal(bf16_bits_to_f64(out), c["out"])
