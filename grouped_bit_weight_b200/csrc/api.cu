@@ -97,7 +97,13 @@ gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
   if (st != GBW_OK) return st;
   if (P == 0) return GBW_OK;
   GroupedProblem pb{x, T, K, w, scale, E, N, offsets, row_to_token, P, out, err};
-  const bool gemv = mode == GBW_MODE_GEMV || (mode == GBW_MODE_AUTO && (P <= 8 || K % 64));
+  const bool fits = gemv_fits(f, pb, sms);
+  if (mode == GBW_MODE_GEMV && !fits)
+    return fail(GBW_ERR_SHAPE, "rows too long for the GEMV's shared-memory ring");
+  if (!fits && K % 64)
+    return fail(GBW_ERR_SHAPE, "rows too long for the GEMV and K % 64 != 0");
+  const bool gemv = mode == GBW_MODE_GEMV ||
+                    (mode == GBW_MODE_AUTO && fits && (P <= 8 || K % 64));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = gemv ? launch_gemv(f, pb, sms, s) : launch_gemm(f, pb, sms, s);
   return e == cudaSuccess ? GBW_OK : launch_error(e);

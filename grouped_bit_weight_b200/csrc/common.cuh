@@ -45,6 +45,8 @@ cudaError_t launch_quantize(Fmt f, const float* w, int64_t rows, int64_t K,
                             uint8_t* codes, void* scale, cudaStream_t s);
 cudaError_t launch_gemv(Fmt f, const GroupedProblem& p, int num_sms,
                         cudaStream_t s);
+// Whether the GEMV's shared-memory ring holds two blocks of rows of length K.
+bool gemv_fits(Fmt f, const GroupedProblem& p, int num_sms);
 cudaError_t launch_gemm(Fmt f, const GroupedProblem& p, int num_sms,
                         cudaStream_t s);
 cudaError_t launch_dgrad(const GroupedProblem& p, int num_sms, cudaStream_t s);
@@ -179,18 +181,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m,
       : "memory");
 }
 
-// Row gather: four rows r0..r3 of a 2-D tensor, columns c0 .. c0+box-1,
-// written as four consecutive box rows at dst (swizzle of the map applies).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m,
-                                            int32_t c0, int32_t r0, int32_t r1,
-                                            int32_t r2, int32_t r3,
-                                            uint64_t* bar) {
+// Bulk (untiled) asynchronous copy of `bytes` contiguous bytes from global
+// to shared memory, completion counted in bytes on `bar`.  Both addresses
+// 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src,
+                                          uint32_t bytes, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::"
-      "complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3), "r"(smem_u32(bar))
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], "
+      "[%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -22,9 +22,19 @@ def test_hand_worked_cases_exact(fmt, mode):
     if mode == "gemm" and c["K"] % 64:
         pytest.skip("the tensor-core path needs K % 64 == 0")
     fn = gbw.gnf4_grouped_gemm if fmt == "nf4" else gbw.gmxfp4_grouped_gemm
+    # the library takes N % 8 == 0: pad each expert with rows whose codes all
+    # decode to zero (NF4 code 7, MXFP4 code 0), which must come out as 0
+    codes, scale = c["codes"], c["scale"]
+    E, N = codes.shape[:2]
+    pad = 8 - N
+    zero = 0x77 if fmt == "nf4" else 0x00
+    codes = np.concatenate([codes, np.full((E, pad) + codes.shape[2:], zero, np.uint8)], axis=1)
+    scale = np.concatenate([scale, np.repeat(scale[:, :1], pad, axis=1)], axis=1)
     x = to_dev(synth.to_bf16_bits(c["x"]))
-    out = fn(x, to_dev(c["codes"]), to_dev(c["scale"]), to_dev(c["offsets"]),
+    out = fn(x, to_dev(codes), to_dev(scale), to_dev(c["offsets"]),
              to_dev(c["row_to_token"]), mode=mode)
     torch.cuda.synchronize()
     assert gbw.device_status() == 0
-    assert np.array_equal(bf16_bits_to_f64(bits(out)), c["out"])
+    got = bf16_bits_to_f64(bits(out))
+    assert np.array_equal(got[:, :N], c["out"])
+    assert np.all(got[:, N:] == 0)
