@@ -192,9 +192,14 @@ def run_ours(args, rank, world, dev):
     out_gu = torch.empty((8, GU.N), dtype=torch.bfloat16, device=dev)
     out_dn = torch.empty((8, DN.N), dtype=torch.bfloat16, device=dev)
 
+    # The expert weights and the routing are written once, before the timed
+    # loop, so every call may overlap the kernel before it (the library reads
+    # x and writes out only after that kernel has finished).
     def step(j):
-        gbw.gnf4_grouped_gemm(x_gu, wgu[0], wgu[1], offs[j], r2ts[j], out=out_gu)
-        gbw.gnf4_grouped_gemm(x_dn, wdn[0], wdn[1], offs[j], None, out=out_dn)
+        gbw.gnf4_grouped_gemm(x_gu, wgu[0], wgu[1], offs[j], r2ts[j], out=out_gu,
+                              overlap_prev=True)
+        gbw.gnf4_grouped_gemm(x_dn, wdn[0], wdn[1], offs[j], None, out=out_dn,
+                              overlap_prev=True)
 
     bytes_gu = gemv_bytes("nf4", 8, GU.N, GU.K, 1)
     bytes_dn = gemv_bytes("nf4", 8, DN.N, DN.K, 8)
@@ -251,7 +256,8 @@ def run_ours(args, rank, world, dev):
     gu_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gu_graph):
         for j in range(N_SETS):
-            gbw.gnf4_grouped_gemm(x_gu, wgu[0], wgu[1], offs[j], r2ts[j], out=out_gu)
+            gbw.gnf4_grouped_gemm(x_gu, wgu[0], wgu[1], offs[j], r2ts[j], out=out_gu,
+                                  overlap_prev=True)
     gu_ms = event_time_ms(torch, gu_graph.replay, 40, stream) / N_SETS
     launches["n"] += 0  # the roofline loop runs outside the timed region
     achieved = bytes_gu / (gu_ms * 1e-3) / 1e9

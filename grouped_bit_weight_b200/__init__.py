@@ -18,7 +18,8 @@ __all__ = [
     "lib", "GbwError", "gnf4_grouped_gemm", "gmxfp4_grouped_gemm",
     "gnf4_grouped_dgrad", "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
     "gmxfp4_quantize", "device_status", "MODE_AUTO", "MODE_GEMM", "MODE_GEMV",
-    "DEVERR_OFFSETS", "DEVERR_TOKEN", "DEVERR_TIMEOUT", "EXPORTS",
+    "DEVERR_OFFSETS", "DEVERR_TOKEN", "DEVERR_TIMEOUT", "FLAG_OVERLAP_PREV",
+    "EXPORTS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,6 +33,7 @@ if not os.path.exists(LIB_PATH):
 lib = C.CDLL(LIB_PATH)
 
 MODE_AUTO, MODE_GEMM, MODE_GEMV = 0, 1, 2
+FLAG_OVERLAP_PREV = 0x100
 DEVERR_OFFSETS, DEVERR_TOKEN, DEVERR_TIMEOUT = 1, 2, 4
 _STATUS = {0: "GBW_OK", 1: "GBW_ERR_NULL", 2: "GBW_ERR_SHAPE",
            3: "GBW_ERR_ALIGN", 4: "GBW_ERR_ARCH", 5: "GBW_ERR_LAUNCH",
@@ -95,7 +97,7 @@ _MODES = {"auto": MODE_AUTO, "gemm": MODE_GEMM, "gemv": MODE_GEMV}
 
 
 def _grouped(fn, where, x, w, scale, scale_dtype, expert_offsets, row_to_token,
-             out, mode, K_div):
+             out, mode, K_div, overlap_prev=False):
     _need(x, "x", torch.bfloat16)
     dev = x.device
     _need(w, "packed weights", torch.uint8, dev)
@@ -118,6 +120,8 @@ def _grouped(fn, where, x, w, scale, scale_dtype, expert_offsets, row_to_token,
     if tuple(out.shape) != (P, N):
         raise ValueError(f"{where}: out must be [{P}, {N}]")
     m = _MODES[mode] if isinstance(mode, str) else int(mode)
+    if overlap_prev:
+        m |= FLAG_OVERLAP_PREV
     with torch.cuda.device(dev):
         _check(fn(_ptr(x), T, K, _ptr(w), _ptr(scale), E, N, _ptr(expert_offsets),
                   _ptr(row_to_token), P, _ptr(out), m, _stream(dev)), where)
@@ -125,22 +129,25 @@ def _grouped(fn, where, x, w, scale, scale_dtype, expert_offsets, row_to_token,
 
 
 def gnf4_grouped_gemm(x, packed, absmax, expert_offsets, row_to_token=None,
-                      out=None, mode="auto"):
+                      out=None, mode="auto", overlap_prev=False):
     """out[P, N] = x[row_to_token] @ W_e^T per expert; NF4 weights
     packed [E, N, K/2] uint8 (high nibble = even k), absmax [E, N, K/64] fp32.
-    P = len(row_to_token), or x's rows when row_to_token is None."""
+    P = len(row_to_token), or x's rows when row_to_token is None.
+    overlap_prev=True promises that packed, absmax, expert_offsets and
+    row_to_token are not written by the kernel launched just before this
+    call on the stream (GBW_FLAG_OVERLAP_PREV)."""
     return _grouped(lib.gnf4_grouped_gemm, "gnf4_grouped_gemm", x, packed,
                     absmax, torch.float32, expert_offsets, row_to_token, out,
-                    mode, 64)
+                    mode, 64, overlap_prev)
 
 
 def gmxfp4_grouped_gemm(x, blocks, scales, expert_offsets, row_to_token=None,
-                        out=None, mode="auto"):
+                        out=None, mode="auto", overlap_prev=False):
     """MXFP4 variant: blocks [E, N, K/32, 16] uint8 (low nibble = even k),
     scales [E, N, K/32] uint8 (e8m0)."""
     return _grouped(lib.gmxfp4_grouped_gemm, "gmxfp4_grouped_gemm", x, blocks,
                     scales, torch.uint8, expert_offsets, row_to_token, out,
-                    mode, 32)
+                    mode, 32, overlap_prev)
 
 
 def gnf4_grouped_dgrad(dy, packed, absmax, expert_offsets, out=None):

@@ -13,6 +13,8 @@ namespace {
 __device__ int g_err_word;
 
 constexpr int kMaxDevices = 64;
+// Experts per call: the kernels keep expert_offsets in shared memory.
+constexpr int32_t kMaxExperts = 4096;
 int* g_err_ptr[kMaxDevices];
 int g_sms[kMaxDevices];
 int g_arch_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
@@ -77,8 +79,11 @@ gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
   if (K > (int64_t)1 << 30 || N > (int64_t)1 << 30 || P > INT32_MAX ||
       T > INT32_MAX || (int64_t)E * N > INT32_MAX)
     return fail(GBW_ERR_SHAPE, "sizes exceed the 32-bit row indices");
-  if (mode < GBW_MODE_AUTO || mode > GBW_MODE_GEMV)
-    return fail(GBW_ERR_SHAPE, "unknown mode");
+  const int32_t flags = mode & ~0xFF;
+  mode &= 0xFF;
+  if (mode < GBW_MODE_AUTO || mode > GBW_MODE_GEMV || (flags & ~GBW_FLAG_OVERLAP_PREV))
+    return fail(GBW_ERR_SHAPE, "unknown mode or flag");
+  if (E > kMaxExperts) return fail(GBW_ERR_SHAPE, "at most 4096 experts");
   if (!offsets || !w || !scale) return fail(GBW_ERR_NULL, "NULL weights or offsets");
   if (P > 0 && (!x || !out)) return fail(GBW_ERR_NULL, "NULL x or out");
   if (!row_to_token && T < P)
@@ -96,7 +101,7 @@ gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
   gbw_status st = device_state(&err, &sms);
   if (st != GBW_OK) return st;
   if (P == 0) return GBW_OK;
-  GroupedProblem pb{x, T, K, w, scale, E, N, offsets, row_to_token, P, out, err};
+  GroupedProblem pb{x, T, K, w, scale, E, N, offsets, row_to_token, P, out, err, flags};
   const bool fits = gemv_fits(f, pb, sms);
   if (mode == GBW_MODE_GEMV && !fits)
     return fail(GBW_ERR_SHAPE, "rows too long for the GEMV's shared-memory ring");
@@ -144,6 +149,7 @@ gbw_status gnf4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
   if (P < 0 || N <= 0 || K <= 0 || E < 1)
     return fail(GBW_ERR_SHAPE, "need P >= 0, N > 0, K > 0, E >= 1");
   if (K % 64 || N % 64) return fail(GBW_ERR_SHAPE, "dgrad needs K % 64 == 0 and N % 64 == 0");
+  if (E > kMaxExperts) return fail(GBW_ERR_SHAPE, "at most 4096 experts");
   if (K > (int64_t)1 << 30 || P > INT32_MAX || (int64_t)E * N > INT32_MAX)
     return fail(GBW_ERR_SHAPE, "sizes exceed the 32-bit row indices");
   if (!packed || !absmax || !expert_offsets) return fail(GBW_ERR_NULL, "NULL weights or offsets");
@@ -157,7 +163,7 @@ gbw_status gnf4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
   gbw_status st = device_state(&err, &sms);
   if (st != GBW_OK) return st;
   if (P == 0) return GBW_OK;
-  GroupedProblem pb{dy, P, K, packed, absmax, E, N, expert_offsets, nullptr, P, dx, err};
+  GroupedProblem pb{dy, P, K, packed, absmax, E, N, expert_offsets, nullptr, P, dx, err, 0};
   cudaError_t e = launch_dgrad(pb, sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GBW_OK : launch_error(e);
 }

@@ -32,6 +32,7 @@ struct GroupedProblem {
   int64_t P;
   uint16_t* out;           // [P, N] bf16 (forward) or dx [P, K] (dgrad)
   int* err;                // device error word
+  int32_t flags;           // GBW_FLAG_* bits of the call
 };
 
 enum class Fmt : int { NF4 = 0, MXFP4 = 1 };
@@ -359,18 +360,42 @@ __device__ __forceinline__ void tmem_load_32x32b_x32(uint32_t taddr,
 // [0, P] (so every row range stays inside the caller's buffers) and flags
 // any change the clamp made.  off_s has E+1 entries.  Whole block; valid
 // offsets (the normal case) are checked in parallel, only invalid ones take
-// the serial clamp.
-__device__ __forceinline__ void load_offsets_clamped(const int32_t* offsets,
-                                                     int32_t E, int64_t P,
-                                                     int32_t* off_s, int* err) {
+// the serial clamp.  Split in two so a kernel can issue the loads first and
+// do other work while they are in flight.
+struct OffsetRegs {
+  int32_t v[2], nxt[2];  // offsets[e] and offsets[e + 1], e = tid, tid + blockDim
+};
+
+__device__ __forceinline__ OffsetRegs prefetch_offsets(const int32_t* offsets,
+                                                       int32_t E) {
+  OffsetRegs r;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int32_t e = (int32_t)(threadIdx.x + k * blockDim.x);
+    r.v[k] = e <= E ? __ldg(offsets + e) : 0;
+    r.nxt[k] = e < E ? __ldg(offsets + e + 1) : 0;
+  }
+  return r;
+}
+
+__device__ __forceinline__ void commit_offsets(const OffsetRegs& r,
+                                               const int32_t* offsets,
+                                               int32_t E, int64_t P,
+                                               int32_t* off_s, int* err) {
   int bad = 0;
-  for (int32_t e = threadIdx.x; e <= E; e += blockDim.x) {
-    const int32_t v = __ldg(offsets + e);
+  auto check = [&](int32_t e, int32_t v, int32_t nxt) {
     off_s[e] = v;
     if (v < 0 || v > (int32_t)P || (e == 0 && v != 0) || (e == E && v != (int32_t)P))
       bad = 1;
-    if (e < E && __ldg(offsets + e + 1) < v) bad = 1;
+    if (e < E && nxt < v) bad = 1;
+  };
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int32_t e = (int32_t)(threadIdx.x + k * blockDim.x);
+    if (e <= E) check(e, r.v[k], r.nxt[k]);
   }
+  for (int32_t e = (int32_t)(threadIdx.x + 2 * blockDim.x); e <= E; e += blockDim.x)
+    check(e, __ldg(offsets + e), e < E ? __ldg(offsets + e + 1) : 0);
   if (__syncthreads_or(bad)) {
     if (threadIdx.x == 0) {
       int32_t prev = 0;
@@ -386,6 +411,23 @@ __device__ __forceinline__ void load_offsets_clamped(const int32_t* offsets,
     }
     __syncthreads();
   }
+}
+
+__device__ __forceinline__ void load_offsets_clamped(const int32_t* offsets,
+                                                     int32_t E, int64_t P,
+                                                     int32_t* off_s, int* err) {
+  commit_offsets(prefetch_offsets(offsets, E), offsets, E, P, off_s, err);
+}
+
+// Programmatic dependent launch: wait until the kernel launched before this
+// one on the stream has completed and its writes are visible (a no-op when
+// this kernel was not launched as a dependent); then let the next kernel on
+// the stream start its own launch.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ts[e] = sum over experts e' < e of tiles(e'), ts[E] = total, where

@@ -57,6 +57,17 @@ typedef enum {
   GBW_MODE_GEMV = 2  /* force the bandwidth GEMV (no tensor cores) */
 } gbw_mode;
 
+/* Flag OR-ed into the mode argument of the grouped forward calls.
+ * GBW_FLAG_OVERLAP_PREV: the caller guarantees that the packed weights, the
+ * scales, expert_offsets and row_to_token of this call are not written by
+ * the kernel launched immediately before it on the same stream (in a MoE
+ * layer they come from the checkpoint and the router, launched earlier).
+ * The bandwidth GEMV then reads them while that kernel is still finishing
+ * (programmatic dependent launch); it reads x and writes out only after the
+ * preceding kernel has completed, with or without the flag.  Passing the
+ * flag when the guarantee does not hold gives undefined results. */
+#define GBW_FLAG_OVERLAP_PREV 0x100
+
 /* Bits of the device error word. */
 #define GBW_DEVERR_OFFSETS 1 /* expert_offsets not 0 <= ... <= P (clamped) */
 #define GBW_DEVERR_TOKEN 2   /* row_to_token[p] outside [0, T) (clamped) */
@@ -77,8 +88,9 @@ typedef enum {
  *   row_to_token   [P] int32 (device) or NULL: routed row p reads x row
  *                  row_to_token[p]; NULL means row p reads x row p (T >= P)
  *   out            [P, N] bf16, row-major, expert-sorted row order
- * Requires K % 64 == 0, N % 8 == 0, E >= 1, and 16-byte aligned x, packed
- * and out.  P == 0 is a no-op.  Experts with no rows cost nothing. */
+ * mode           a gbw_mode, optionally OR-ed with GBW_FLAG_OVERLAP_PREV
+ * Requires K % 64 == 0, N % 8 == 0, 1 <= E <= 4096, and 16-byte aligned x,
+ * packed and out.  P == 0 is a no-op.  Experts with no rows cost nothing. */
 GBW_API gbw_status gnf4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
                              const uint8_t* packed, const float* absmax,
                              int32_t E, int64_t N,

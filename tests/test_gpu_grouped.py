@@ -234,3 +234,33 @@ def test_repeatable_and_path_independent(fmt, layer, tokens):
         assert torch.equal(a.view(torch.int16), ref.view(torch.int16))
         assert torch.equal(b.view(torch.int16), ref.view(torch.int16))
     assert gbw.device_status() == 0
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
+def test_overlap_prev_chain_reads_x_after_the_previous_kernel(fmt):
+    """Programmatic dependent launch: with overlap_prev=True the GEMV may read
+    weights and routing while the kernel before it still runs, but x only
+    after it.  Here each call's x is the previous call's output, so reading
+    x early would use stale values; 50 chained launches must give exactly
+    the bits of the same calls run one at a time."""
+    E, N, K = 4, 512, 512
+    codes, scale, _ = packed_weights(fmt, E, N, K, 0.05, 51)
+    off = np.array([0, 2, 4, 6, 8], np.int32)  # 8 routed rows, 2 per expert
+    fn = FWD[fmt]
+    dc, ds, do = to_dev(codes), to_dev(scale), to_dev(off)
+    x0 = to_dev(synth.to_bf16_bits(synth.normal((8, K), 52)))
+
+    def chain(overlap, sync_each):
+        x = x0
+        for _ in range(50):
+            x = fn(x, dc, ds, do, None, mode="gemv", overlap_prev=overlap)
+            if sync_each:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return bits(x)
+
+    ref = chain(False, True)
+    got = chain(True, False)
+    assert gbw.device_status() == 0
+    assert np.array_equal(got, ref)
+    assert np.any(ref != 0)  # the chain did not decay to all zeros
