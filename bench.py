@@ -63,6 +63,30 @@ def gemm_flops(P, N, K):
     return 2.0 * P * N * K
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank times its own replica on its own
+    device; the job takes as long as the slowest one (a MAX all-reduce of
+    one number, on the process group's backend: NCCL on GPUs, gloo in the
+    CPU tests)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(bytes_per_rank_step: float, steps: int, world: int, ms_max: float,
+             scale: float = 1e9) -> float:
+    """Whole-job throughput: every rank processed `steps` steps of
+    `bytes_per_rank_step`, all done when the slowest rank is."""
+    return world * bytes_per_rank_step * steps / (ms_max * 1e-3) / scale
+
+
 # ---------------------------------------------------------------- clocks
 
 class Clocks:
@@ -242,14 +266,10 @@ def run_ours(args, rank, world, dev):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = t0.elapsed_time(t1)
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     launches["n"] += 2 * args.steps
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
     ms_per_step = ms / args.steps
-    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+    value = job_rate(bytes_step, args.steps, world, ms)
 
     # dominant kernel: the gate_up GEMV alone, back to back in a graph of
     # one launch per expert set; average device time per launch
@@ -270,7 +290,7 @@ def run_ours(args, rank, world, dev):
                 "launch_ms": round(gu_ms, 5), "peak_source": peak_kind}
 
     # e2e: host buffers, copies inside the timed region, public API calls
-    e2e = measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step)
+    e2e = measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step, world)
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
@@ -305,7 +325,7 @@ def load_traffic(name):
         return None
 
 
-def measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step):
+def measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step, world=1):
     """Same decode layer through the public API with host buffers: every step
     copies its inputs (x, offsets, row map) from pinned host memory and
     reads both outputs back; one synchronisation per step."""
@@ -341,13 +361,17 @@ def measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step):
     for j in range(32):
         one(j % N_SETS)
     torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
     t = time.perf_counter()
     for i in range(n):
         one(i % N_SETS)
-    dt = time.perf_counter() - t
-    return {"value": round(bytes_step * n / dt / 1e9, 2), "unit": "GB/s",
+    ms = max_over_ranks((time.perf_counter() - t) * 1e3, world, dev)
+    return {"value": round(job_rate(bytes_step, n, world, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": n,
-            "timing": "host wall clock around steps that each end in a stream sync"}
+            "timing": "host wall clock around steps that each end in a stream "
+                      "sync; max over ranks"}
 
 
 def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):

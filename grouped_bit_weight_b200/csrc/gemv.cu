@@ -38,34 +38,36 @@
 namespace gbw {
 namespace {
 
-__constant__ float kNF4g[16] = {
-    -1.0f,
-    -0.6961928009986877f,
-    -0.5250730514526367f,
-    -0.39491748809814453f,
-    -0.28444138169288635f,
-    -0.18477343022823334f,
-    -0.09105003625154495f,
-    0.0f,
-    0.07958029955625534f,
-    0.16093020141124725f,
-    0.24611230194568634f,
-    0.33791524171829224f,
-    0.44070982933044434f,
-    0.5626170039176941f,
-    0.7229568362236023f,
-    1.0f,
-};
-__constant__ float kE2M1g[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
-
 constexpr int kThreads = 384;  // 12 warps: up to 168 registers a thread
 constexpr int kWarps = kThreads / 32;
 constexpr int kLutBytes = 256 * 256;  // 256 entries x 256-byte rows
 
+// Codebook value of code q, from immediates (a select tree, no memory
+// access: a table in constant memory costs a cold miss on every launch).
+// NF4: the 16 QLoRA levels; MXFP4: OCP e2m1 (bit 3 = sign).
 __device__ __forceinline__ float code_value(Fmt F, uint32_t q) {
-  if (F == Fmt::NF4) return kNF4g[q];
-  const float m = kE2M1g[q & 7u];
-  return (q & 8u) ? -m : m;
+  if (F == Fmt::NF4) {
+    const float lo8[8] = {-1.0f, -0.6961928009986877f, -0.5250730514526367f,
+                          -0.39491748809814453f, -0.28444138169288635f,
+                          -0.18477343022823334f, -0.09105003625154495f, 0.0f};
+    const float hi8[8] = {0.07958029955625534f, 0.16093020141124725f,
+                          0.24611230194568634f, 0.33791524171829224f,
+                          0.44070982933044434f, 0.5626170039176941f,
+                          0.7229568362236023f, 1.0f};
+    float r = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      r = (q == (uint32_t)i) ? lo8[i] : r;
+      r = (q == (uint32_t)(i + 8)) ? hi8[i] : r;
+    }
+    return r;
+  }
+  const uint32_t m = q & 7u;
+  // e2m1 magnitude: exponent field m >> 1 (bias 1), mantissa bit m & 1
+  const float mag = (m < 2u) ? 0.5f * (float)m
+                             : __int_as_float((int)((126u + (m >> 1)) << 23)) *
+                                   (1.0f + 0.5f * (float)(m & 1u));
+  return (q & 8u) ? -mag : mag;
 }
 
 __device__ __forceinline__ float e8m0_f32(uint32_t s) {
