@@ -316,11 +316,18 @@ def run_ours(args, rank, world, dev):
 
 
 def load_traffic(name):
-    """DRAM bytes per launch from the committed ncu summary, if present."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of `name` from the committed ncu summary
+    (profiles/traffic.json), or None when absent or when the kernel sources
+    have changed since the capture (their sha256 no longer matches)."""
+    import hashlib
     try:
-        with open(p) as f:
-            return json.load(f).get(name)
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            ent = json.load(f)[name]
+        d = hashlib.sha256()
+        for rel in ent["sources"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                d.update(f.read())
+        return ent["bytes"] if d.hexdigest() == ent["source_sha256"] else None
     except Exception:
         return None
 
