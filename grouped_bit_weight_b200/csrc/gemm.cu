@@ -7,32 +7,30 @@
 // in HBM.
 //
 // B200 design (one persistent CTA per SM, 16 warps):
-//   tile  = 128 weight rows (MMA M) x up to 256 routed rows (MMA N) x K,
-//           i.e. the matmul runs as out^T = W x^T ("swap AB"), so an expert
-//           with few routed rows gets a narrow MMA N instead of a padded M;
-//   warps 2-3   the tile's x rows -> 128B-swizzled smem ring (4 stages of
-//               64 K): one 2-D TMA tile per stage when routed row p reads x
-//               row p; 16-byte cp.async from 64 threads when rows are
-//               gathered through row_to_token (one TMA tile::gather4 per four
-//               rows measured ~4x slower: the TMA front end serialises them)
+//   tile  = 128 weight rows (MMA M) x up to 256 routed rows (MMA N) x K: the
+//           matmul runs as out^T = W x^T ("swap AB"), so an expert with few
+//           routed rows gets a narrow MMA N instead of a padded M.  On B200 a
+//           single-CTA tcgen05.mma (M = 128, K = 16) costs about the same
+//           issue time whatever its N (measured: ~244 cycles from N = 64 to
+//           256), so tiles use the widest N the routed rows allow;
 //   warps 4-11  decode: each thread owns one weight row; per 64-K stage it
-//               loads its 32 packed bytes (one 32-byte sector) and the block
-//               scale straight from global memory, two of its stages ahead,
-//               builds the block's bf16 table and decodes with byte
-//               permutes, then stores the 64 bf16 as one
-//               128-byte row of the 128B-swizzled A tile (4-stage smem ring);
-//               two groups of four warps take alternate stages
-//   warp 1      one thread issues tcgen05.mma (A and B from smem, fp32
-//               accumulator in TMEM) and tcgen05.commit
-//   warps 12-15 epilogue: tcgen05.ld the 128 x N accumulator, round to bf16,
-//               transpose through smem, 16-byte stores of out rows
-// Tensor memory holds two 128 x 256 fp32 accumulators, so the epilogue of
-// one tile overlaps the mainloop of the next.
-// (Staging the packed weights through a TMA ring of 128 x 32-byte boxes was
-// tried first: the decode warps on the three sub-partitions without the
-// issuing warp occasionally read bytes that differed from global memory
-// after the ring's full barrier had completed.  Per-thread sector loads
-// avoid the ring and measured exact.)
+//               takes its 32 packed bytes and block scale (loaded from global
+//               memory three of its stages ahead), builds the block's bf16
+//               table, decodes with byte permutes and stores the 64 bf16 as
+//               one 128-byte row of the 128B-swizzled, K-major A tile
+//               (4-stage ring); two groups of four warps take alternate stages;
+//   warp 2      activations, identity rows: one 2-D TMA tile (64 K x 256
+//               rows, 128B swizzle) per stage into a 4-stage ring;
+//   warps 0,2,3 activations gathered through row_to_token: eight consecutive
+//               lanes copy one row's 128 bytes of a stage with 16-byte
+//               cp.async, so each warp instruction moves four whole rows;
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (A and B from
+//               shared memory, fp32 accumulator in TMEM) and tcgen05.commit;
+//   warps 12-15 epilogue: tcgen05.ld 32 accumulator columns (routed rows) of
+//               the warp's 32 weight rows, round to bf16, transpose 32 x 32
+//               through shared memory and write 16-byte pieces of output rows.
+// Tensor memory holds two 128 x 256 fp32 accumulators, so the epilogue of one
+// tile overlaps the mainloop of the next.
 // Scheduler: tiles (expert, 128-row weight tile, 256-row token tile) with
 // zero-row experts skipped, enumerated from expert_offsets by every CTA and
 // dealt round-robin (token tiles innermost, so CTAs running at the same time
@@ -53,18 +51,19 @@ constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 
 constexpr int kXStageBytes = BT * BK * 2;      // 32 KB
 constexpr int kAStageBytes = BM * BK * 2;      // 16 KB
+constexpr int kGatherThreads = 96;             // warps 0, 2, 3
 constexpr int kEpiRowBytes = 80;               // 64 B of data + 16 B pad
 constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
 
 struct Smem {
-  // byte offsets inside the dynamic shared memory block
+  // byte offsets inside the dynamic shared memory block (1024-aligned base)
   static constexpr int x = 0;
   static constexpr int a = x + XS * kXStageBytes;
-  static constexpr int epi = a + AS * kAStageBytes;
+  static constexpr int epi = a + AS * kAStageBytes;  // epilogue transpose
   static constexpr int bars = epi + 4 * kEpiWarpBytes;
   static constexpr int nbars = 2 * XS + 2 * AS + 5;
-  static constexpr int misc = bars + nbars * 8;  // tmem base, abort flag
-  static constexpr int tables = misc + 16;       // offsets[E+1], tile_start[E+1]
+  static constexpr int misc = bars + nbars * 8;      // tmem base, abort flag
+  static constexpr int tables = misc + 16;           // offsets[E+1], tile_start[E+1]
 };
 
 struct TileInfo {
@@ -72,8 +71,7 @@ struct TileInfo {
 };
 
 __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
-                                              const int32_t* ts, int32_t E,
-                                              int32_t ntn) {
+                                              const int32_t* ts, int32_t E) {
   int32_t lo = 0, hi = E - 1;  // last e with ts[e] <= t
   while (lo < hi) {
     int32_t mid = (lo + hi + 1) >> 1;
@@ -88,7 +86,6 @@ __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
   ti.n0 = nt * BM;
   ti.p0 = off[lo] + mt * BT;
   ti.nv = min(BT, cnt - mt * BT);
-  (void)ntn;
   return ti;
 }
 
@@ -96,7 +93,7 @@ template <Fmt F>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte alignment for the 128B-swizzled activation tiles
+  // 1024-byte alignment for the 128B-swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::bars);
@@ -117,18 +114,14 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
   const int64_t K = pb.K, N = pb.N;
   const int NK = (int)(K / BK);
   const int32_t ntn = (int32_t)((N + BM - 1) / BM);
+  const bool gathered = pb.row_to_token != nullptr;
 
   if (threadIdx.x == 0) {
-    const uint32_t xcount = pb.row_to_token ? 64u : 1u;  // 64 copy threads or one TMA
+    // TMA: one arrival plus bytes; gather: every gather thread arrives
+    const uint32_t xcount = gathered ? (uint32_t)kGatherThreads : 1u;
     for (int i = 0; i < XS; ++i) { mbar_init(&x_full[i], xcount); mbar_init(&x_empty[i], 1); }
-    for (int i = 0; i < AS; ++i) {
-      mbar_init(&a_full[i], 4);
-      mbar_init(&a_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
-    }
+    for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
     mbar_init(mma_done, 1);
     *abort = 0;
     fence_barrier_init();
@@ -137,7 +130,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 2 && lane == 0) tma_prefetch_desc(&tmx);
+  if (warp == 2 && lane == 0 && !gathered) tma_prefetch_desc(&tmx);
   load_offsets_clamped(pb.offsets, E, pb.P, off_s, pb.err);  // has __syncthreads
   tile_prefix(off_s, E, BT, ntn, ts_s);
   tc_fence_before();
@@ -146,15 +139,15 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
   const uint32_t tmem = *tmem_slot;
   const int64_t ntiles = ts_s[E];
 
-  if (warp == 2 || warp == 3) {
+  if (warp == 0 || warp == 2 || warp == 3) {
     // ---------------- activation producer ----------------
     uint32_t g = 0;
     bool ok = true;
-    if (pb.row_to_token == nullptr) {
+    if (!gathered) {
       // routed row p reads x row p: one 2-D TMA tile (64 K x 256 rows) per stage
       if (warp == 2 && lane == 0) {
         for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-          const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
+          const TileInfo ti = tile_info(t, off_s, ts_s, E);
           for (int kb = 0; kb < NK; ++kb, ++g) {
             const uint32_t s = g % XS, ph = (g / XS) & 1u;
             if (!(ok = mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err))) break;
@@ -167,51 +160,43 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
             mbar_drain(&x_full[i % XS], (i / XS) & 1u);
       }
     } else {
-      // gathered rows: 64 threads copy 16-byte chunks with cp.async, placing
-      // chunk c of row r at (c ^ (r % 8)) -- the 128-byte swizzle the MMA's
-      // descriptor expects.  cp.async writes through the generic proxy, so a
-      // thread publishes stage g only after its own copies of g have landed
-      // (wait_group) and a proxy fence; XS - 1 stages stay in flight.
-      constexpr int kLag = XS - 1;  // < XS, or the producer would wait on itself
-      const int pt = (warp - 2) * 32 + lane;  // rows pt, pt+64, pt+128, pt+192
-      uint32_t pub = 0;                       // stages published so far
-      auto publish_upto = [&](uint32_t upto) {
-        for (; pub < upto; ++pub) mbar_arrive(&x_full[pub % XS]);
-      };
+      // Gathered rows.  Lane l of gather warp w copies 16-byte chunk (l & 7)
+      // of rows 4w + (l >> 3) + 12i: eight lanes cover one row's 128 bytes,
+      // so a warp instruction moves four whole rows.  Chunk c of row r lands
+      // at (c ^ (r % 8)) -- the 128-byte swizzle the MMA's descriptor
+      // expects.  Each thread keeps the token ids of its rows in registers
+      // (no barrier between the gather warps, so an aborted wait in one
+      // cannot strand the others) and ends each stage with an mbarrier
+      // arrival that fires when its copies land, so a stage is published as
+      // soon as its bytes are in shared memory.  cp.async writes through the
+      // generic proxy: the MMA thread fences the proxies after its wait.
+      constexpr int kRows = (BT + 11) / 12;     // rows per thread
+      const int gw = warp == 0 ? 0 : warp - 1;  // gather warp 0..2
+      const int chunk = lane & 7;
+      const int r0 = 4 * gw + (lane >> 3);
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
-        const uint16_t* src[4];
+        const TileInfo ti = tile_info(t, off_s, ts_s, E);
+        int32_t tk[kRows];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = pt + 64 * i;
-          src[i] = r < ti.nv
-                       ? pb.x + (int64_t)token_of_row(pb.row_to_token, ti.p0 + r, pb.T, pb.err) * K
-                       : nullptr;
+        for (int i = 0; i < kRows; ++i) {
+          const int r = r0 + 12 * i;
+          tk[i] = r < ti.nv ? token_of_row(pb.row_to_token, ti.p0 + r, pb.T, pb.err) : -1;
         }
         for (int kb = 0; kb < NK; ++kb, ++g) {
           const uint32_t s = g % XS, ph = (g / XS) & 1u;
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err)))) break;
           const uint32_t dst = smem_u32(smem + Smem::x + s * kXStageBytes);
+          const uint16_t* xk = pb.x + kb * BK + chunk * 8;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (!src[i]) continue;
-            const int r = pt + 64 * i;
-            const uint16_t* sp = src[i] + kb * BK;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              cp_async_16(dst + r * 128 + ((c ^ (r & 7)) << 4), sp + c * 8);
+          for (int i = 0; i < kRows; ++i) {
+            const int r = r0 + 12 * i;
+            if (tk[i] >= 0)
+              cp_async_16(dst + r * 128 + ((chunk ^ (r & 7)) << 4), xk + (int64_t)tk[i] * K);
           }
-          cp_async_commit();
-          if (g + 1 > (uint32_t)kLag) {
-            cp_async_wait_group<kLag>();  // stage g - kLag has landed
-            fence_proxy_async();
-            publish_upto(g + 1 - kLag);
-          }
+          cp_async_arrive_noinc(&x_full[s]);
         }
       }
-      cp_async_wait_all();
-      fence_proxy_async();
-      if (ok) publish_upto(g);
+      cp_async_wait_all();  // nothing may still be landing when the CTA exits
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -221,7 +206,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
       const uint32_t xbase = smem_u32(smem + Smem::x);
       const uint32_t abase = smem_u32(smem + Smem::a);
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
-        const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
+        const TileInfo ti = tile_info(t, off_s, ts_s, E);
         const uint32_t nmma = (uint32_t)((ti.nv + 15) & ~15);
         const uint32_t idesc = make_idesc_bf16(BM, nmma, 0, 0);
         const uint32_t ab = it & 1u;
@@ -232,6 +217,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
           const uint32_t xs = g % XS, as = g % AS;
           if (!(ok = mbar_wait(&a_full[as], (g / AS) & 1u, abort, pb.err))) break;
           if (!(ok = mbar_wait(&x_full[xs], (g / XS) & 1u, abort, pb.err))) break;
+          if (gathered) fence_proxy_async();  // cp.async landed via the generic proxy
           tc_fence_after();
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
@@ -257,8 +243,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
     const int64_t my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const uint32_t total = (uint32_t)(my_tiles * NK);
     // The row's 32 packed bytes and its block scale for stage g are read
-    // from global memory four stages (two of this group's) ahead of their
-    // use, so their latency overlaps decode work.
+    // from global memory six stages (three of this group's) ahead of use.
     struct Pf { uint4 q0, q1; uint32_t sc; };
     int64_t pf_tile = -1, pf_wrow = 0;
     bool pf_valid = false;
@@ -270,7 +255,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
       const int64_t ti_idx = g / NK;
       if (ti_idx != pf_tile) {
         pf_tile = ti_idx;
-        const TileInfo ti = tile_info(blockIdx.x + ti_idx * gridDim.x, off_s, ts_s, E, ntn);
+        const TileInfo ti = tile_info(blockIdx.x + ti_idx * gridDim.x, off_s, ts_s, E);
         pf_valid = ti.n0 + m < N;
         pf_wrow = (int64_t)ti.e * N + ti.n0 + m;
       }
@@ -286,11 +271,12 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
             reinterpret_cast<const uint8_t*>(pb.scale) + pf_wrow * (K / 32) + 2 * kb));
       return f;
     };
-    Pf f0 = fetch(grp), f1 = fetch(grp + 2);
+    Pf f0 = fetch(grp), f1 = fetch(grp + 2), f2 = fetch(grp + 4);
     for (uint32_t g = grp; g < total; g += 2) {
       const Pf cur = f0;
       f0 = f1;
-      f1 = fetch(g + 4);
+      f1 = f2;
+      f2 = fetch(g + 6);
       const uint32_t sv = cur.sc;
       const uint32_t as = g % AS, aph = (g / AS) & 1u;
       const uint32_t P[8] = {cur.q0.x, cur.q0.y, cur.q0.z, cur.q0.w,
@@ -321,11 +307,15 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
     }
   } else if (warp >= 12) {
     // ---------------- epilogue ----------------
+    // Thread t of warp q holds output column n0 + 32q + t for 32 routed rows
+    // per TMEM chunk; a 32 x 32 bf16 transpose through shared memory turns
+    // that into 64 contiguous bytes of one output row per thread, written
+    // with four 16-byte stores.
     const uint32_t q = (uint32_t)warp & 3u;
     uint8_t* stage = smem + Smem::epi + q * kEpiWarpBytes;
     uint32_t it = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-      const TileInfo ti = tile_info(t, off_s, ts_s, E, ntn);
+      const TileInfo ti = tile_info(t, off_s, ts_s, E);
       const uint32_t ab = it & 1u;
       const uint32_t tlane = tmem + ((q * 32u) << 16) + ab * 256u;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (it >> 1) & 1u, abort, pb.err));
@@ -341,7 +331,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
-        // thread = output column ncol0+lane, r[j] = routed row c*32+j
+        // thread = output column ncol0 + lane, r[j] = routed row c*32 + j
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           *reinterpret_cast<uint16_t*>(stage + j * kEpiRowBytes + lane * 2) =
