@@ -37,6 +37,7 @@ constexpr int LS = 4;     // load ring stages (dy + packed)
 constexpr int DS = 3;     // decoded-B ring stages
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
+static_assert(BR == 64, "the MMA issuer unrolls four 16-row steps per stage");
 
 constexpr int kAStageBytes = BM * BR * 2;   // 16 KB
 constexpr int kWStageBytes = BR * BN / 2;   // 8 KB
@@ -151,8 +152,10 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
     if (lane == 0) {
       uint32_t g = 0, it = 0;
       bool ok = true;
-      const uint32_t ldbase = smem_u32(smem + Smem::ld);
-      const uint32_t bbase = smem_u32(smem + Smem::b);
+      // descriptors advance by 64-bit adds (start address in 16-byte units):
+      // nothing but the MMAs runs between them in this thread
+      const uint64_t adesc0 = make_sdesc_sw128(smem_u32(smem + Smem::ld), 16, 1024);
+      const uint64_t bdesc0 = make_sdesc_sw128(smem_u32(smem + Smem::b), 1024, 4096);
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
         const DTile d = dtile_info(t, off_s, ts_s, E);
         const uint32_t nmma = (uint32_t)min((int64_t)BN, K - d.k0);
@@ -166,14 +169,12 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
           if (!(ok = mbar_wait(&ld_full[ls], (g / LS) & 1u, abort, pb.err))) break;
           if (!(ok = mbar_wait(&b_full[bs], (g / DS) & 1u, abort, pb.err))) break;
           tc_fence_after();
-#pragma unroll
-          for (int j = 0; j < BR / 16; ++j) {
-            const uint64_t adesc =
-                make_sdesc_sw128(ldbase + ls * kLStageBytes + j * 32, 16, 1024);
-            const uint64_t bdesc =
-                make_sdesc_sw128(bbase + bs * kBStageBytes + j * 8192, 1024, 4096);
-            tc_mma_ss(dacc, adesc, bdesc, idesc, (ks | j) != 0);
-          }
+          const uint64_t ad = adesc0 + (uint64_t)((ls * kLStageBytes) >> 4);
+          const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes) >> 4);
+          tc_mma_ss(dacc, ad, bd, idesc, ks != 0);
+          tc_mma_ss(dacc, ad + 2, bd + 512, idesc, 1u);   // A +32 B, B +8 KB: next 16 n
+          tc_mma_ss(dacc, ad + 4, bd + 1024, idesc, 1u);
+          tc_mma_ss(dacc, ad + 6, bd + 1536, idesc, 1u);
           tc_commit(&ld_empty[ls]);
           tc_commit(&b_empty[bs]);
         }

@@ -48,6 +48,7 @@ constexpr int XS = 4;     // activation ring stages
 constexpr int AS = 4;     // decoded-weight (A operand) ring stages
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
+static_assert(BK == 64, "the MMA issuer unrolls four K = 16 steps per stage");
 
 constexpr int kXStageBytes = BT * BK * 2;      // 32 KB
 constexpr int kAStageBytes = BM * BK * 2;      // 16 KB
@@ -200,11 +201,16 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // One thread keeps the tensor core fed: the loop holds no descriptor
+    // arithmetic beyond 64-bit adds (the start-address field counts 16-byte
+    // units), because everything this thread executes between MMAs adds to
+    // their issue time (measured: a 128 x 256 x 16 MMA takes 128 cycles when
+    // issued back to back, ~240 with descriptors rebuilt around it).
     if (lane == 0) {
       uint32_t g = 0, it = 0;
       bool ok = true;
-      const uint32_t xbase = smem_u32(smem + Smem::x);
-      const uint32_t abase = smem_u32(smem + Smem::a);
+      const uint64_t xdesc0 = make_sdesc_sw128(smem_u32(smem + Smem::x), 16, 1024);
+      const uint64_t adesc0 = make_sdesc_sw128(smem_u32(smem + Smem::a), 16, 1024);
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
         const TileInfo ti = tile_info(t, off_s, ts_s, E);
         const uint32_t nmma = (uint32_t)((ti.nv + 15) & ~15);
@@ -219,12 +225,12 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
           if (!(ok = mbar_wait(&x_full[xs], (g / XS) & 1u, abort, pb.err))) break;
           if (gathered) fence_proxy_async();  // cp.async landed via the generic proxy
           tc_fence_after();
-#pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t adesc = make_sdesc_sw128(abase + as * kAStageBytes + j * 32, 16, 1024);
-            const uint64_t bdesc = make_sdesc_sw128(xbase + xs * kXStageBytes + j * 32, 16, 1024);
-            tc_mma_ss(dacc, adesc, bdesc, idesc, (kb | j) != 0);
-          }
+          const uint64_t ad = adesc0 + (uint64_t)((as * kAStageBytes) >> 4);
+          const uint64_t bd = xdesc0 + (uint64_t)((xs * kXStageBytes) >> 4);
+          tc_mma_ss(dacc, ad, bd, idesc, kb != 0);
+          tc_mma_ss(dacc, ad + 2, bd + 2, idesc, 1u);  // +32 bytes: next 16 K
+          tc_mma_ss(dacc, ad + 4, bd + 4, idesc, 1u);
+          tc_mma_ss(dacc, ad + 6, bd + 6, idesc, 1u);
           tc_commit(&x_empty[xs]);
           tc_commit(&a_empty[as]);
         }
@@ -247,6 +253,11 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
     struct Pf { uint4 q0, q1; uint32_t sc; };
     int64_t pf_tile = -1, pf_wrow = 0;
     bool pf_valid = false;
+    // NF4 absmax rows are K/64 floats; when that is a multiple of four a
+    // single 16-byte load brings the scales of four stages (cached below)
+    const bool sc4 = F == Fmt::NF4 && (K / 64) % 4 == 0;
+    int64_t sc4_key = -1;
+    float4 sc4_val = make_float4(0.f, 0.f, 0.f, 0.f);
     auto fetch = [&](uint32_t g) -> Pf {
       Pf f;
       f.q0 = f.q1 = make_uint4(0u, 0u, 0u, 0u);
@@ -264,7 +275,16 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
       const uint4* wp = reinterpret_cast<const uint4*>(pb.w + pf_wrow * (K / 2) + kb * (BK / 2));
       f.q0 = __ldg(wp);
       f.q1 = __ldg(wp + 1);
-      if (F == Fmt::NF4)
+      if (F == Fmt::NF4 && sc4) {
+        const int64_t key = pf_wrow * (K / 256) + (kb >> 2);
+        if (key != sc4_key) {
+          sc4_key = key;
+          sc4_val = __ldg(reinterpret_cast<const float4*>(pb.scale) + key);
+        }
+        const int sel = kb & 3;
+        const float v = sel == 0 ? sc4_val.x : sel == 1 ? sc4_val.y : sel == 2 ? sc4_val.z : sc4_val.w;
+        f.sc = __float_as_uint(v);
+      } else if (F == Fmt::NF4)
         f.sc = __float_as_uint(__ldg(reinterpret_cast<const float*>(pb.scale) + pf_wrow * (K / 64) + kb));
       else
         f.sc = __ldg(reinterpret_cast<const uint16_t*>(
@@ -337,15 +357,17 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
           *reinterpret_cast<uint16_t*>(stage + j * kEpiRowBytes + lane * 2) =
               __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[j])));
         __syncwarp();
-        const int row = c * 32 + lane;  // routed row within the tile
-        if (row < ti.nv) {
-          uint16_t* dst = pb.out + (int64_t)(ti.p0 + row) * N + ncol0;
+        // four lanes write one routed row's 64 bytes, so each store
+        // instruction covers eight whole row segments (full 32-byte sectors)
+        const int sub = lane & 3;              // 16-byte piece of the row
+        const bool subok = ncol0 + sub * 8 < N;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (ncol0 + v * 8 < N)
-              reinterpret_cast<uint4*>(dst)[v] =
-                  *reinterpret_cast<const uint4*>(stage + lane * kEpiRowBytes + v * 16);
-          }
+        for (int v = 0; v < 4; ++v) {
+          const int rr = (lane >> 2) + 8 * v;  // row within the chunk
+          const int row = c * 32 + rr;         // routed row within the tile
+          if (row < ti.nv && subok)
+            *reinterpret_cast<uint4*>(pb.out + (int64_t)(ti.p0 + row) * N + ncol0 + sub * 8) =
+                *reinterpret_cast<const uint4*>(stage + rr * kEpiRowBytes + sub * 16);
         }
         __syncwarp();
       }
