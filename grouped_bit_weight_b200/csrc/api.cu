@@ -14,7 +14,7 @@ __device__ int g_err_word;
 
 constexpr int kMaxDevices = 64;
 // Experts per call: the kernels keep expert_offsets in shared memory.
-constexpr int32_t kMaxExperts = 2048;
+constexpr int32_t kMaxExperts = 1024;
 int* g_err_ptr[kMaxDevices];
 int g_sms[kMaxDevices];
 int g_arch_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
@@ -83,7 +83,7 @@ gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
   mode &= 0xFF;
   if (mode < GBW_MODE_AUTO || mode > GBW_MODE_GEMV || (flags & ~GBW_FLAG_OVERLAP_PREV))
     return fail(GBW_ERR_SHAPE, "unknown mode or flag");
-  if (E > kMaxExperts) return fail(GBW_ERR_SHAPE, "at most 2048 experts");
+  if (E > kMaxExperts) return fail(GBW_ERR_SHAPE, "at most 1024 experts");
   if (!offsets || !w || !scale) return fail(GBW_ERR_NULL, "NULL weights or offsets");
   if (P > 0 && (!x || !out)) return fail(GBW_ERR_NULL, "NULL x or out");
   if (!row_to_token && T < P)
@@ -149,7 +149,7 @@ gbw_status gnf4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
   if (P < 0 || N <= 0 || K <= 0 || E < 1)
     return fail(GBW_ERR_SHAPE, "need P >= 0, N > 0, K > 0, E >= 1");
   if (K % 64 || N % 64) return fail(GBW_ERR_SHAPE, "dgrad needs K % 64 == 0 and N % 64 == 0");
-  if (E > kMaxExperts) return fail(GBW_ERR_SHAPE, "at most 2048 experts");
+  if (E > kMaxExperts) return fail(GBW_ERR_SHAPE, "at most 1024 experts");
   if (K > (int64_t)1 << 30 || P > INT32_MAX || (int64_t)E * N > INT32_MAX)
     return fail(GBW_ERR_SHAPE, "sizes exceed the 32-bit row indices");
   if (!packed || !absmax || !expert_offsets) return fail(GBW_ERR_NULL, "NULL weights or offsets");

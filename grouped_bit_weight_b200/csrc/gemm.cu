@@ -46,23 +46,26 @@ constexpr int BT = 256;   // routed rows per tile (max MMA N)
 constexpr int BK = 64;    // K per stage
 constexpr int XS = 4;     // activation ring stages
 constexpr int AS = 4;     // decoded-weight (A operand) ring stages
+constexpr int WG = 2;     // packed-weight ring stages per decode group
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 static_assert(BK == 64, "the MMA issuer unrolls four K = 16 steps per stage");
 
 constexpr int kXStageBytes = BT * BK * 2;      // 32 KB
 constexpr int kAStageBytes = BM * BK * 2;      // 16 KB
+constexpr int kWStageBytes = BM * BK / 2;      // 4 KB: 128 rows x 32 packed bytes
 constexpr int kGatherThreads = 96;             // warps 0, 2, 3
-constexpr int kEpiRowBytes = 80;               // 64 B of data + 16 B pad
+constexpr int kEpiRowBytes = 64;               // one transposed row (read 4 lanes a row: no conflicts)
 constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
 
 struct Smem {
   // byte offsets inside the dynamic shared memory block (1024-aligned base)
   static constexpr int x = 0;
   static constexpr int a = x + XS * kXStageBytes;
-  static constexpr int epi = a + AS * kAStageBytes;  // epilogue transpose
+  static constexpr int w = a + AS * kAStageBytes;    // packed weights, 2 groups
+  static constexpr int epi = w + 2 * WG * kWStageBytes;  // epilogue transpose
   static constexpr int bars = epi + 4 * kEpiWarpBytes;
-  static constexpr int nbars = 2 * XS + 2 * AS + 5;
+  static constexpr int nbars = 2 * XS + 2 * AS + 4 * WG + 5;
   static constexpr int misc = bars + nbars * 8;      // tmem base, abort flag
   static constexpr int tables = misc + 16;           // offsets[E+1], tile_start[E+1]
 };
@@ -92,7 +95,8 @@ __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
 
 template <Fmt F>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
+gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
+            const __grid_constant__ CUtensorMap tmw) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128B-swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -102,7 +106,9 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
   uint64_t* x_empty = x_full + XS;
   uint64_t* a_full = x_empty + XS;
   uint64_t* a_empty = a_full + AS;
-  uint64_t* acc_full = a_empty + AS;   // [2]
+  uint64_t* w_full = a_empty + AS;     // [2][WG]
+  uint64_t* w_empty = w_full + 2 * WG; // [2][WG]
+  uint64_t* acc_full = w_empty + 2 * WG;  // [2]
   uint64_t* acc_empty = acc_full + 2;  // [2]
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc);
@@ -122,6 +128,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
     const uint32_t xcount = gathered ? (uint32_t)kGatherThreads : 1u;
     for (int i = 0; i < XS; ++i) { mbar_init(&x_full[i], xcount); mbar_init(&x_empty[i], 1); }
     for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < 2 * WG; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], 4); }
     for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
     mbar_init(mma_done, 1);
     *abort = 0;
@@ -132,6 +139,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
     tmem_relinquish();
   }
   if (warp == 2 && lane == 0 && !gathered) tma_prefetch_desc(&tmx);
+  if ((warp == 4 || warp == 8) && lane == 0) tma_prefetch_desc(&tmw);
   load_offsets_clamped(pb.offsets, E, pb.P, off_s, pb.err);  // has __syncthreads
   tile_prefix(off_s, E, BT, ntn, ts_s);
   tc_fence_before();
@@ -242,65 +250,82 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
     }
   } else if (warp >= 4 && warp < 12) {
     // ---------------- decode ----------------
-    const uint32_t grp = (uint32_t)(warp - 4) >> 2;  // takes stages g with g % 2 == grp
+    // Group grp (warps 4-7 or 8-11) takes the stages g = grp + 2h.  The
+    // packed bytes of a stage (128 rows x 32 bytes) arrive by TMA into the
+    // group's own 2-slot ring: the first lane of the group issues stage h+2
+    // once all four warps have read slot h, so no decode thread issues a
+    // global load for them (per-thread loads of 32 bytes from 32 different
+    // rows were the kernel's bottleneck).
+    const uint32_t grp = (uint32_t)(warp - 4) >> 2;
     const uint32_t q = (uint32_t)warp & 3u;
     const int m = (int)(q * 32 + lane);              // weight row in tile
     const int mr = m & 7;                            // row inside its 8-row atom
+    const bool issuer = q == 0 && lane == 0;
+    uint64_t* wf = w_full + grp * WG;
+    uint64_t* we = w_empty + grp * WG;
+    uint8_t* wring = smem + Smem::w + grp * WG * kWStageBytes;
     const int64_t my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const uint32_t total = (uint32_t)(my_tiles * NK);
-    // The row's 32 packed bytes and its block scale for stage g are read
-    // from global memory six stages (three of this group's) ahead of use.
-    struct Pf { uint4 q0, q1; uint32_t sc; };
-    int64_t pf_tile = -1, pf_wrow = 0;
-    bool pf_valid = false;
-    // NF4 absmax rows are K/64 floats; when that is a multiple of four a
-    // single 16-byte load brings the scales of four stages (cached below)
-    const bool sc4 = F == Fmt::NF4 && (K / 64) % 4 == 0;
-    int64_t sc4_key = -1;
-    float4 sc4_val = make_float4(0.f, 0.f, 0.f, 0.f);
-    auto fetch = [&](uint32_t g) -> Pf {
-      Pf f;
-      f.q0 = f.q1 = make_uint4(0u, 0u, 0u, 0u);
-      f.sc = 0u;
-      if (g >= total) return f;
-      const int64_t ti_idx = g / NK;
-      if (ti_idx != pf_tile) {
-        pf_tile = ti_idx;
-        const TileInfo ti = tile_info(blockIdx.x + ti_idx * gridDim.x, off_s, ts_s, E);
-        pf_valid = ti.n0 + m < N;
-        pf_wrow = (int64_t)ti.e * N + ti.n0 + m;
+    const uint32_t nh = total > grp ? (total - grp + 1) / 2 : 0;  // this group's stages
+    // tile of stage g, cached (stages advance monotonically)
+    int64_t c_tile = -1;
+    TileInfo c_ti{};
+    auto tile_of = [&](uint32_t g) -> const TileInfo& {
+      const int64_t idx = g / NK;
+      if (idx != c_tile) {
+        c_tile = idx;
+        c_ti = tile_info(blockIdx.x + idx * gridDim.x, off_s, ts_s, E);
       }
-      if (!pf_valid) return f;
-      const int kb = (int)(g % NK);
-      const uint4* wp = reinterpret_cast<const uint4*>(pb.w + pf_wrow * (K / 2) + kb * (BK / 2));
-      f.q0 = __ldg(wp);
-      f.q1 = __ldg(wp + 1);
-      if (F == Fmt::NF4 && sc4) {
-        const int64_t key = pf_wrow * (K / 256) + (kb >> 2);
-        if (key != sc4_key) {
-          sc4_key = key;
-          sc4_val = __ldg(reinterpret_cast<const float4*>(pb.scale) + key);
-        }
-        const int sel = kb & 3;
-        const float v = sel == 0 ? sc4_val.x : sel == 1 ? sc4_val.y : sel == 2 ? sc4_val.z : sc4_val.w;
-        f.sc = __float_as_uint(v);
-      } else if (F == Fmt::NF4)
-        f.sc = __float_as_uint(__ldg(reinterpret_cast<const float*>(pb.scale) + pf_wrow * (K / 64) + kb));
-      else
-        f.sc = __ldg(reinterpret_cast<const uint16_t*>(
-            reinterpret_cast<const uint8_t*>(pb.scale) + pf_wrow * (K / 32) + 2 * kb));
-      return f;
+      return c_ti;
     };
-    Pf f0 = fetch(grp), f1 = fetch(grp + 2), f2 = fetch(grp + 4);
-    for (uint32_t g = grp; g < total; g += 2) {
-      const Pf cur = f0;
-      f0 = f1;
-      f1 = f2;
-      f2 = fetch(g + 6);
-      const uint32_t sv = cur.sc;
+    uint32_t issued = 0;  // group stages issued so far (issuer lane)
+    auto issue_w = [&](uint32_t h) {  // TMA of group stage h into slot h % WG
+      const uint32_t g = grp + 2 * h;
+      const TileInfo ti = tile_of(g);
+      const int kb = (int)(g % NK);
+      issued = h + 1;
+      mbar_arrive_expect_tx(&wf[h % WG], kWStageBytes);
+      tma_load_2d(wring + (h % WG) * kWStageBytes, &tmw, kb * (BK / 2),
+                  (int32_t)((int64_t)ti.e * N + ti.n0), &wf[h % WG]);
+    };
+    // the block scale of stage g for row m (a plain load; its value is not
+    // touched until the stage it belongs to)
+    auto scale_of = [&](uint32_t g) -> uint32_t {
+      const TileInfo& ti = tile_of(g);
+      if (ti.n0 + m >= N) return 0u;
+      const int64_t wrow = (int64_t)ti.e * N + ti.n0 + m;
+      const int kb = (int)(g % NK);
+      if (F == Fmt::NF4)
+        return __float_as_uint(__ldg(reinterpret_cast<const float*>(pb.scale) + wrow * (K / 64) + kb));
+      return __ldg(reinterpret_cast<const uint16_t*>(
+          reinterpret_cast<const uint8_t*>(pb.scale) + wrow * (K / 32) + 2 * kb));
+    };
+    if (issuer)
+      for (uint32_t h = 0; h < WG && h < nh; ++h) issue_w(h);
+    // The loop is unrolled by two with one scale register per half: the
+    // scale of stage h + 2 is loaded right after stage h and not read until
+    // then (a queue rotated by register copies would wait on each load one
+    // stage after issuing it).
+    bool ok = true;
+    uint32_t h = 0;  // next group stage to consume
+    auto stage = [&](uint32_t sv) -> bool {
+      const uint32_t g = grp + 2 * h;
+      const uint32_t ws = h % WG, wph = (h / WG) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&wf[ws], wph, abort, pb.err))) return false;
+      const uint8_t* wrow_s = wring + ws * kWStageBytes + m * 32;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(wrow_s);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(wrow_s + 16);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&we[ws]);
+      bool good = true;
+      if (issuer && h + WG < nh) {
+        // slot ws is free once all four warps of the group have read it
+        good = mbar_wait(&we[ws], wph, abort, pb.err);
+        if (good) issue_w(h + WG);
+      }
+      if (!__all_sync(0xffffffffu, good)) return false;
       const uint32_t as = g % AS, aph = (g / AS) & 1u;
-      const uint32_t P[8] = {cur.q0.x, cur.q0.y, cur.q0.z, cur.q0.w,
-                             cur.q1.x, cur.q1.y, cur.q1.z, cur.q1.w};
+      const uint32_t P[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
       uint32_t o[32];
       if (F == Fmt::NF4) {
         const Planes tb = nf4_planes(__uint_as_float(sv));
@@ -314,7 +339,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
 #pragma unroll
         for (int i = 4; i < 8; ++i) decode_word<false>(P[i], t1, &o[4 * i]);
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], aph ^ 1u, abort, pb.err))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], aph ^ 1u, abort, pb.err))) return false;
       // row m of the K-major, 128B-swizzled A tile: chunk c at (c ^ (m % 8))
       uint8_t* dst = smem + Smem::a + as * kAStageBytes + m * 128;
 #pragma unroll
@@ -324,7 +349,25 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx) {
       fence_proxy_async();  // generic-proxy stores -> tensor core reads
       __syncwarp();
       if (lane == 0) mbar_arrive(&a_full[as]);
+      return true;
+    };
+    auto scale_h = [&](uint32_t hh) -> uint32_t { return hh < nh ? scale_of(grp + 2 * hh) : 0u; };
+    uint32_t sA = scale_h(0), sB = scale_h(1);
+    while (h < nh) {
+      if (!(ok = stage(sA))) break;
+      ++h;
+      sA = scale_h(h + 1);
+      if (h >= nh) break;
+      if (!(ok = stage(sB))) break;
+      ++h;
+      sB = scale_h(h + 1);
     }
+    // After an abort, copies this group issued but did not consume must
+    // land before the CTA exits (shared memory is still their target).
+    // Stage h (where the group stopped) onwards are still in flight; every
+    // earlier one was waited for.
+    if (issuer && !ok)
+      for (uint32_t d = h; d < issued; ++d) mbar_drain(&wf[d % WG], (d / WG) & 1u);
   } else if (warp >= 12) {
     // ---------------- epilogue ----------------
     // Thread t of warp q holds output column n0 + 32q + t for 32 routed rows
@@ -434,12 +477,19 @@ cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
                               (uint64_t)pb.K, (uint64_t)(pb.T > 0 ? pb.T : 1),
                               (uint64_t)pb.K * 2, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
+  // packed weights [E*N rows, K/2 bytes]: boxes of 32 bytes (one 64-K stage)
+  // x 128 rows; rows past E*N read as zeros
+  CUtensorMap tmw;
+  e = make_map_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.w, (uint64_t)pb.K / 2,
+                  (uint64_t)pb.E * (uint64_t)pb.N, (uint64_t)pb.K / 2, BK / 2, BM,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (e != cudaSuccess) return e;
   const size_t smem = gemm_smem_bytes(pb.E);
   auto k = (f == Fmt::NF4) ? gemm_kernel<Fmt::NF4> : gemm_kernel<Fmt::MXFP4>;
   e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<num_sms, kThreads, smem, s>>>(pb, tmx);
+  k<<<num_sms, kThreads, smem, s>>>(pb, tmx, tmw);
   return cudaGetLastError();
 }
 

@@ -89,7 +89,7 @@ typedef enum {
  *                  row_to_token[p]; NULL means row p reads x row p (T >= P)
  *   out            [P, N] bf16, row-major, expert-sorted row order
  * mode           a gbw_mode, optionally OR-ed with GBW_FLAG_OVERLAP_PREV
- * Requires K % 64 == 0, N % 8 == 0, 1 <= E <= 2048, and 16-byte aligned x,
+ * Requires K % 64 == 0, N % 8 == 0, 1 <= E <= 1024, and 16-byte aligned x,
  * packed and out.  P == 0 is a no-op.  Experts with no rows cost nothing. */
 GBW_API gbw_status gnf4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
                              const uint8_t* packed, const float* absmax,

@@ -52,7 +52,7 @@ def test_host_validation_needs_no_gpu(fn):
     assert _call(fn, P=-1) == SHAPE
     assert _call(fn, mode=7) == SHAPE
     assert _call(fn, mode=0x200) == SHAPE     # unknown flag bit
-    assert _call(fn, E=2049) == SHAPE         # more experts than the kernels hold
+    assert _call(fn, E=1025) == SHAPE         # more experts than the kernels hold
     assert _call(fn, T=2, P=4) == SHAPE       # identity rows need T >= P
     assert _call(fn, off=0) == NULL
     assert _call(fn, w=0) == NULL
