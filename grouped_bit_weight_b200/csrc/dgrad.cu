@@ -227,13 +227,16 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
       const uint8_t* wst = smem + Smem::ld + ls * kLStageBytes + kAStageBytes + n * 128;
       const uint4 q0 = *reinterpret_cast<const uint4*>(wst + (((2 * j) ^ rr) << 4));
       const uint4 q1 = *reinterpret_cast<const uint4*>(wst + (((2 * j + 1) ^ rr) << 4));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ld_empty[ls]);
       uint32_t o[32];
       const uint32_t P[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
       const Planes tb = nf4_planes(a);
 #pragma unroll
       for (int i = 0; i < 8; ++i) decode_word<true>(P[i], tb, &o[4 * i]);
+      // release the slab only once the decode has consumed what was loaded
+      // from it: the refill is an async-proxy (TMA) write and must not
+      // overtake shared-memory loads still in flight
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ld_empty[ls]);
       if (!__all_sync(0xffffffffu, mbar_wait(&b_empty[bs], ((g / DS) & 1u) ^ 1u, abort, pb.err))) break;
       if (jvalid) {
         // K-row n of atom (n/8, j): 128 bytes, chunk c at (c ^ rr)

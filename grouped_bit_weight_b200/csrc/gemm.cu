@@ -9,18 +9,20 @@
 // B200 design (one persistent CTA per SM, 16 warps):
 //   tile  = 128 weight rows (MMA M) x up to 256 routed rows (MMA N) x K: the
 //           matmul runs as out^T = W x^T ("swap AB"), so an expert with few
-//           routed rows gets a narrow MMA N instead of a padded M.  On B200 a
-//           single-CTA tcgen05.mma (M = 128, K = 16) costs about the same
-//           issue time whatever its N (measured: ~244 cycles from N = 64 to
-//           256), so tiles use the widest N the routed rows allow;
-//   warps 4-11  decode: each thread owns one weight row; per 64-K stage it
-//               takes its 32 packed bytes and block scale (loaded from global
-//               memory three of its stages ahead), builds the block's bf16
-//               table, decodes with byte permutes and stores the 64 bf16 as
-//               one 128-byte row of the 128B-swizzled, K-major A tile
-//               (4-stage ring); two groups of four warps take alternate stages;
+//           routed rows gets a narrow MMA N instead of a padded M;
+//   warps 4-11  decode, two groups of four warps taking alternate 64-K
+//               stages.  A stage's packed bytes (128 rows x 32 bytes) arrive
+//               by TMA into the group's 2-slot ring; a tile's scales (128
+//               consecutive rows of one expert, one contiguous range) arrive
+//               by one bulk copy into a double buffer.  Each thread owns one
+//               weight row: it builds the block's bf16 table, decodes with
+//               byte permutes and stores the 64 bf16 as one 128-byte row of
+//               the 128B-swizzled, K-major A tile (one slot per group).
+//               These warps bound the kernel by the instructions they issue,
+//               so their loop does no per-stage divisions or global loads;
 //   warp 2      activations, identity rows: one 2-D TMA tile (64 K x 256
-//               rows, 128B swizzle) per stage into a 4-stage ring;
+//               rows, 128B swizzle) per stage into a 4-stage ring (32-row
+//               boxes for a partial tile);
 //   warps 0,2,3 activations gathered through row_to_token: eight consecutive
 //               lanes copy one row's 128 bytes of a stage with 16-byte
 //               cp.async, so each warp instruction moves four whole rows;
@@ -28,7 +30,7 @@
 //               shared memory, fp32 accumulator in TMEM) and tcgen05.commit;
 //   warps 12-15 epilogue: tcgen05.ld 32 accumulator columns (routed rows) of
 //               the warp's 32 weight rows, round to bf16, transpose 32 x 32
-//               through shared memory and write 16-byte pieces of output rows.
+//               through shared memory and write whole 64-byte row segments.
 // Tensor memory holds two 128 x 256 fp32 accumulators, so the epilogue of one
 // tile overlaps the mainloop of the next.
 // Scheduler: tiles (expert, 128-row weight tile, 256-row token tile) with
@@ -45,7 +47,8 @@ constexpr int BM = 128;   // weight rows per tile (MMA M)
 constexpr int BT = 256;   // routed rows per tile (max MMA N)
 constexpr int BK = 64;    // K per stage
 constexpr int XS = 4;     // activation ring stages
-constexpr int AS = 4;     // decoded-weight (A operand) ring stages
+constexpr int AS = 2;     // decoded-weight (A operand) ring stages: one per decode group
+static_assert(AS % 2 == 0, "the two decode groups own alternate A slots");
 constexpr int WG = 2;     // packed-weight ring stages per decode group
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
@@ -54,6 +57,7 @@ static_assert(BK == 64, "the MMA issuer unrolls four K = 16 steps per stage");
 constexpr int kXStageBytes = BT * BK * 2;      // 32 KB
 constexpr int kAStageBytes = BM * BK * 2;      // 16 KB
 constexpr int kWStageBytes = BM * BK / 2;      // 4 KB: 128 rows x 32 packed bytes
+constexpr int kScaleBuf = 16 * 1024;           // one tile's scales (double buffered)
 constexpr int kGatherThreads = 96;             // warps 0, 2, 3
 constexpr int kEpiRowBytes = 64;               // one transposed row (read 4 lanes a row: no conflicts)
 constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
@@ -63,9 +67,10 @@ struct Smem {
   static constexpr int x = 0;
   static constexpr int a = x + XS * kXStageBytes;
   static constexpr int w = a + AS * kAStageBytes;    // packed weights, 2 groups
-  static constexpr int epi = w + 2 * WG * kWStageBytes;  // epilogue transpose
+  static constexpr int sc = w + 2 * WG * kWStageBytes;   // tile scales, 2 buffers
+  static constexpr int epi = sc + 2 * kScaleBuf;         // epilogue transpose
   static constexpr int bars = epi + 4 * kEpiWarpBytes;
-  static constexpr int nbars = 2 * XS + 2 * AS + 4 * WG + 5;
+  static constexpr int nbars = 2 * XS + 2 * AS + 4 * WG + 4 + 5;
   static constexpr int misc = bars + nbars * 8;      // tmem base, abort flag
   static constexpr int tables = misc + 16;           // offsets[E+1], tile_start[E+1]
 };
@@ -96,7 +101,9 @@ __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
 template <Fmt F>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
-            const __grid_constant__ CUtensorMap tmw) {
+            const __grid_constant__ CUtensorMap tmx32,
+            const __grid_constant__ CUtensorMap tmw, const int srow,
+            const int tile_scales) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128B-swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -108,7 +115,9 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
   uint64_t* a_empty = a_full + AS;
   uint64_t* w_full = a_empty + AS;     // [2][WG]
   uint64_t* w_empty = w_full + 2 * WG; // [2][WG]
-  uint64_t* acc_full = w_empty + 2 * WG;  // [2]
+  uint64_t* sc_full = w_empty + 2 * WG;  // [2]
+  uint64_t* sc_empty = sc_full + 2;      // [2]
+  uint64_t* acc_full = sc_empty + 2;     // [2]
   uint64_t* acc_empty = acc_full + 2;  // [2]
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc);
@@ -129,6 +138,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     for (int i = 0; i < XS; ++i) { mbar_init(&x_full[i], xcount); mbar_init(&x_empty[i], 1); }
     for (int i = 0; i < AS; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < 2 * WG; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], 4); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&sc_full[i], 1); mbar_init(&sc_empty[i], 8); }
     for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
     mbar_init(mma_done, 1);
     *abort = 0;
@@ -138,7 +148,10 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 2 && lane == 0 && !gathered) tma_prefetch_desc(&tmx);
+  if (warp == 2 && lane == 0 && !gathered) {
+    tma_prefetch_desc(&tmx);
+    tma_prefetch_desc(&tmx32);
+  }
   if ((warp == 4 || warp == 8) && lane == 0) tma_prefetch_desc(&tmw);
   load_offsets_clamped(pb.offsets, E, pb.P, off_s, pb.err);  // has __syncthreads
   tile_prefix(off_s, E, BT, ntn, ts_s);
@@ -153,15 +166,26 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     uint32_t g = 0;
     bool ok = true;
     if (!gathered) {
-      // routed row p reads x row p: one 2-D TMA tile (64 K x 256 rows) per stage
+      // routed row p reads x row p: one 2-D TMA tile (64 K x 256 rows) per
+      // stage; a tile with fewer rows loads only the 32-row boxes it uses
+      // (activation reads from L2 bound the kernel, and most experts end in
+      // a partial tile)
       if (warp == 2 && lane == 0) {
         for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
           const TileInfo ti = tile_info(t, off_s, ts_s, E);
           for (int kb = 0; kb < NK; ++kb, ++g) {
             const uint32_t s = g % XS, ph = (g / XS) & 1u;
             if (!(ok = mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err))) break;
-            mbar_arrive_expect_tx(&x_full[s], kXStageBytes);
-            tma_load_2d(smem + Smem::x + s * kXStageBytes, &tmx, kb * BK, ti.p0, &x_full[s]);
+            uint8_t* dst = smem + Smem::x + s * kXStageBytes;
+            if (ti.nv == BT) {
+              mbar_arrive_expect_tx(&x_full[s], kXStageBytes);
+              tma_load_2d(dst, &tmx, kb * BK, ti.p0, &x_full[s]);
+            } else {
+              const int nb = (ti.nv + 31) >> 5;  // 32-row boxes of 4 KB
+              mbar_arrive_expect_tx(&x_full[s], (uint32_t)nb * (32 * BK * 2));
+              for (int b = 0; b < nb; ++b)
+                tma_load_2d(dst + b * (32 * BK * 2), &tmx32, kb * BK, ti.p0 + 32 * b, &x_full[s]);
+            }
           }
         }
         if (*abort)
@@ -252,79 +276,142 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     // ---------------- decode ----------------
     // Group grp (warps 4-7 or 8-11) takes the stages g = grp + 2h.  The
     // packed bytes of a stage (128 rows x 32 bytes) arrive by TMA into the
-    // group's own 2-slot ring: the first lane of the group issues stage h+2
-    // once all four warps have read slot h, so no decode thread issues a
-    // global load for them (per-thread loads of 32 bytes from 32 different
-    // rows were the kernel's bottleneck).
+    // group's own ring: the first lane of the group issues stage h + WG once
+    // all four warps have read slot h.  A tile's scales (128 consecutive
+    // rows of one expert: one contiguous range) arrive by one bulk copy
+    // into a double buffer, issued a tile ahead by the first lane of group
+    // 0; shapes whose tile scales do not fit load each stage's scale per
+    // thread instead, two stages ahead.
+    // These warps bound the kernel by the instructions they issue, so the
+    // loop keeps its bookkeeping incremental: a cursor per look-ahead
+    // distance (the stage being decoded, the scale load, the weight TMA)
+    // steps two stages at a time and looks a tile up only when it enters a
+    // new one -- no divisions per stage.
     const uint32_t grp = (uint32_t)(warp - 4) >> 2;
     const uint32_t q = (uint32_t)warp & 3u;
     const int m = (int)(q * 32 + lane);              // weight row in tile
     const int mr = m & 7;                            // row inside its 8-row atom
-    const bool issuer = q == 0 && lane == 0;
+    const bool issuer = q == 0 && lane == 0;         // packed-weight TMA
+    const bool sc_issuer = issuer && grp == 0;       // tile-scale copies
     uint64_t* wf = w_full + grp * WG;
     uint64_t* we = w_empty + grp * WG;
     uint8_t* wring = smem + Smem::w + grp * WG * kWStageBytes;
     const int64_t my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const uint32_t total = (uint32_t)(my_tiles * NK);
     const uint32_t nh = total > grp ? (total - grp + 1) / 2 : 0;  // this group's stages
-    // tile of stage g, cached (stages advance monotonically)
-    int64_t c_tile = -1;
-    TileInfo c_ti{};
-    auto tile_of = [&](uint32_t g) -> const TileInfo& {
-      const int64_t idx = g / NK;
-      if (idx != c_tile) {
-        c_tile = idx;
-        c_ti = tile_info(blockIdx.x + idx * gridDim.x, off_s, ts_s, E);
+    // first weight row (e * N + n0) of local tile tl
+    auto tile_row = [&](int64_t tl) -> int64_t {
+      const TileInfo ti = tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E);
+      return (int64_t)ti.e * N + ti.n0;
+    };
+    auto tile_n0 = [&](int64_t tl) -> int32_t {
+      return tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E).n0;
+    };
+    // cursor: local tile tl and stage kb of group stage h; step() = h + 1
+    struct Cursor {
+      int64_t tl;
+      int kb;
+    };
+    auto at = [&](uint32_t hh) -> Cursor {  // once per cursor, at the start
+      const uint32_t g = grp + 2 * hh;
+      return Cursor{(int64_t)(g / NK), (int)(g % NK)};
+    };
+    auto step = [&](Cursor& c) -> bool {  // true when it enters a new tile
+      c.kb += 2;
+      if (c.kb < NK) return false;
+      do { c.kb -= NK; ++c.tl; } while (c.kb >= NK);
+      return true;
+    };
+    // weight TMA cursor (issuer lane only)
+    Cursor wc = at(0);
+    int32_t wrow0 = nh ? (int32_t)tile_row(wc.tl) : 0;
+    uint32_t issued = 0;  // group stages whose packed bytes were requested
+    auto issue_w = [&]() {  // the stage at wc into slot issued % WG
+      const uint32_t slot = issued % WG;
+      ++issued;
+      mbar_arrive_expect_tx(&wf[slot], kWStageBytes);
+      tma_load_2d(wring + slot * kWStageBytes, &tmw, wc.kb * (BK / 2), wrow0, &wf[slot]);
+      if (step(wc) && issued < nh) wrow0 = (int32_t)tile_row(wc.tl);
+    };
+    // one tile's scales: rows e*N + n0 .. +127 (clipped at the end of the
+    // array); rows past the expert are read but never used
+    const int64_t total_rows = (int64_t)E * N;
+    int64_t sc_issued = 0;
+    auto issue_sc = [&](int64_t tl) {
+      const int64_t row0 = tile_row(tl);
+      const int64_t rows = min((int64_t)BM, total_rows - row0);
+      const uint32_t bytes = (uint32_t)(rows * srow);
+      sc_issued = tl + 1;
+      mbar_arrive_expect_tx(&sc_full[tl & 1], bytes);
+      bulk_load(smem + Smem::sc + (tl & 1) * kScaleBuf,
+                reinterpret_cast<const uint8_t*>(pb.scale) + row0 * srow, bytes, &sc_full[tl & 1]);
+    };
+    // per-thread scale loads (when tile scales do not fit): cursor two
+    // stages ahead of the decode and this thread's scale row of its tile
+    Cursor lc = at(0);
+    const uint8_t* lrow = nullptr;  // scale row of weight row m, or null past N
+    const int sbytes = F == Fmt::NF4 ? 4 : 2;  // scale bytes per stage
+    auto lrow_of = [&](int64_t tl) -> const uint8_t* {
+      const int32_t n0 = tile_n0(tl);
+      if (n0 + m >= N) return nullptr;
+      return reinterpret_cast<const uint8_t*>(pb.scale) + (tile_row(tl) + m) * (int64_t)srow;
+    };
+    auto scale_next = [&](uint32_t hh) -> uint32_t {  // the scale of stage hh (= lc)
+      uint32_t v = 0;
+      if (hh < nh) {
+        if (lrow) {
+          if (F == Fmt::NF4)
+            v = __ldg(reinterpret_cast<const uint32_t*>(lrow + lc.kb * sbytes));
+          else
+            v = __ldg(reinterpret_cast<const uint16_t*>(lrow + lc.kb * sbytes));
+        }
+        if (step(lc) && hh + 1 < nh) lrow = lrow_of(lc.tl);
       }
-      return c_ti;
-    };
-    uint32_t issued = 0;  // group stages issued so far (issuer lane)
-    auto issue_w = [&](uint32_t h) {  // TMA of group stage h into slot h % WG
-      const uint32_t g = grp + 2 * h;
-      const TileInfo ti = tile_of(g);
-      const int kb = (int)(g % NK);
-      issued = h + 1;
-      mbar_arrive_expect_tx(&wf[h % WG], kWStageBytes);
-      tma_load_2d(wring + (h % WG) * kWStageBytes, &tmw, kb * (BK / 2),
-                  (int32_t)((int64_t)ti.e * N + ti.n0), &wf[h % WG]);
-    };
-    // the block scale of stage g for row m (a plain load; its value is not
-    // touched until the stage it belongs to)
-    auto scale_of = [&](uint32_t g) -> uint32_t {
-      const TileInfo& ti = tile_of(g);
-      if (ti.n0 + m >= N) return 0u;
-      const int64_t wrow = (int64_t)ti.e * N + ti.n0 + m;
-      const int kb = (int)(g % NK);
-      if (F == Fmt::NF4)
-        return __float_as_uint(__ldg(reinterpret_cast<const float*>(pb.scale) + wrow * (K / 64) + kb));
-      return __ldg(reinterpret_cast<const uint16_t*>(
-          reinterpret_cast<const uint8_t*>(pb.scale) + wrow * (K / 32) + 2 * kb));
+      return v;
     };
     if (issuer)
-      for (uint32_t h = 0; h < WG && h < nh; ++h) issue_w(h);
-    // The loop is unrolled by two with one scale register per half: the
-    // scale of stage h + 2 is loaded right after stage h and not read until
-    // then (a queue rotated by register copies would wait on each load one
-    // stage after issuing it).
+      while (issued < WG && issued < nh) issue_w();
+    if (sc_issuer && tile_scales)
+      for (int64_t t = 0; t < 2 && t < my_tiles; ++t) issue_sc(t);
+    uint32_t sA = 0, sB = 0;
+    if (!tile_scales) {
+      if (nh) lrow = lrow_of(lc.tl);
+      sA = scale_next(0);
+      sB = scale_next(1);
+    }
     bool ok = true;
-    uint32_t h = 0;  // next group stage to consume
+    uint32_t h = 0;  // next group stage
+    Cursor dc = at(0);  // the stage being decoded
+    auto publish_slot = [&](uint32_t slot) {
+      fence_proxy_async();  // generic-proxy stores -> tensor core reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[slot]);
+    };
+    uint32_t ws = 0, wph = 0;              // packed-weight slot and parity of stage h
+    uint32_t as = grp, aph = 0;            // A slot and parity of stage h
     auto stage = [&](uint32_t sv) -> bool {
-      const uint32_t g = grp + 2 * h;
-      const uint32_t ws = h % WG, wph = (h / WG) & 1u;
+      const int64_t tl = dc.tl;
+      const int kb = dc.kb;
+      if (tile_scales && kb < 2) {  // the group's first stage of this tile
+        if (!__all_sync(0xffffffffu, mbar_wait(&sc_full[tl & 1], (uint32_t)(tl >> 1) & 1u, abort, pb.err)))
+          return false;
+        // the other buffer: its tile (tl - 1) must be released by both groups
+        bool good = true;
+        if (sc_issuer && tl >= 1 && tl + 1 < my_tiles) {
+          good = mbar_wait(&sc_empty[(tl + 1) & 1], (uint32_t)((tl - 1) >> 1) & 1u, abort, pb.err);
+          if (good) issue_sc(tl + 1);
+        }
+        if (!__all_sync(0xffffffffu, good)) return false;
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&wf[ws], wph, abort, pb.err))) return false;
       const uint8_t* wrow_s = wring + ws * kWStageBytes + m * 32;
       const uint4 q0 = *reinterpret_cast<const uint4*>(wrow_s);
       const uint4 q1 = *reinterpret_cast<const uint4*>(wrow_s + 16);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&we[ws]);
-      bool good = true;
-      if (issuer && h + WG < nh) {
-        // slot ws is free once all four warps of the group have read it
-        good = mbar_wait(&we[ws], wph, abort, pb.err);
-        if (good) issue_w(h + WG);
+      if (tile_scales) {
+        const uint8_t* sb = smem + Smem::sc + (tl & 1) * kScaleBuf + m * srow + kb * sbytes;
+        sv = F == Fmt::NF4 ? *reinterpret_cast<const uint32_t*>(sb)
+                           : (uint32_t)*reinterpret_cast<const uint16_t*>(sb);
       }
-      if (!__all_sync(0xffffffffu, good)) return false;
-      const uint32_t as = g % AS, aph = (g / AS) & 1u;
       const uint32_t P[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
       uint32_t o[32];
       if (F == Fmt::NF4) {
@@ -339,6 +426,21 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
 #pragma unroll
         for (int i = 4; i < 8; ++i) decode_word<false>(P[i], t1, &o[4 * i]);
       }
+      // Release the packed-weight slot (and, after the tile's last stage,
+      // the scale buffer) only now that the decode has consumed the values
+      // loaded from them: the refill is an async-proxy write, and releasing
+      // right after issuing the shared-memory loads let the refill of the
+      // issuing warp's own slot overtake loads still in flight.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&we[ws]);
+      if (tile_scales && kb + 2 >= NK && lane == 0) mbar_arrive(&sc_empty[tl & 1]);
+      bool good = true;
+      if (issuer && issued < nh) {
+        // slot ws is free once all four warps of the group have used it
+        good = mbar_wait(&we[ws], wph, abort, pb.err);
+        if (good) issue_w();
+      }
+      if (!__all_sync(0xffffffffu, good)) return false;
       if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], aph ^ 1u, abort, pb.err))) return false;
       // row m of the K-major, 128B-swizzled A tile: chunk c at (c ^ (m % 8))
       uint8_t* dst = smem + Smem::a + as * kAStageBytes + m * 128;
@@ -346,28 +448,33 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(dst + ((c ^ mr) << 4)) =
             make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-      fence_proxy_async();  // generic-proxy stores -> tensor core reads
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[as]);
+      publish_slot(as);
+      // next group stage: slots advance by one (weights) and two (A)
+      if (++ws == WG) { ws = 0; wph ^= 1u; }
+      as += 2;
+      if (as >= AS) { as -= AS; aph ^= 1u; }
+      step(dc);
       return true;
     };
-    auto scale_h = [&](uint32_t hh) -> uint32_t { return hh < nh ? scale_of(grp + 2 * hh) : 0u; };
-    uint32_t sA = scale_h(0), sB = scale_h(1);
+    // unrolled by two with one scale register per half: the scale of stage
+    // h + 2 is loaded right after stage h and not read until then (a queue
+    // rotated by register copies would wait on each load right away)
     while (h < nh) {
       if (!(ok = stage(sA))) break;
       ++h;
-      sA = scale_h(h + 1);
+      if (!tile_scales) sA = scale_next(h + 1);
       if (h >= nh) break;
       if (!(ok = stage(sB))) break;
       ++h;
-      sB = scale_h(h + 1);
+      if (!tile_scales) sB = scale_next(h + 1);
     }
-    // After an abort, copies this group issued but did not consume must
+    // After an abort, copies this group requested but did not consume must
     // land before the CTA exits (shared memory is still their target).
-    // Stage h (where the group stopped) onwards are still in flight; every
-    // earlier one was waited for.
     if (issuer && !ok)
       for (uint32_t d = h; d < issued; ++d) mbar_drain(&wf[d % WG], (d / WG) & 1u);
+    if (sc_issuer && !ok)
+      for (int64_t t = (sc_issued > 2 ? sc_issued - 2 : 0); t < sc_issued; ++t)
+        mbar_drain(&sc_full[t & 1], (uint32_t)(t >> 1) & 1u);
   } else if (warp >= 12) {
     // ---------------- epilogue ----------------
     // Thread t of warp q holds output column n0 + 32q + t for 32 routed rows
@@ -463,6 +570,9 @@ cudaError_t make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+static_assert(1024 + Smem::tables + 8 * (1024 + 1) <= 232448,
+              "shared memory for 1024 experts exceeds the 227 KB a CTA can have");
+
 size_t gemm_smem_bytes(int32_t E) {
   return 1024 + Smem::tables + sizeof(int32_t) * 2 * (size_t)(E + 1);
 }
@@ -477,6 +587,11 @@ cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
                               (uint64_t)pb.K, (uint64_t)(pb.T > 0 ? pb.T : 1),
                               (uint64_t)pb.K * 2, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
+  CUtensorMap tmx32;  // the same rows in boxes of 32, for partial tiles
+  e = make_map_2d(&tmx32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pb.x,
+                  (uint64_t)pb.K, (uint64_t)(pb.T > 0 ? pb.T : 1),
+                  (uint64_t)pb.K * 2, BK, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
   // packed weights [E*N rows, K/2 bytes]: boxes of 32 bytes (one 64-K stage)
   // x 128 rows; rows past E*N read as zeros
   CUtensorMap tmw;
@@ -484,12 +599,21 @@ cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
                   (uint64_t)pb.E * (uint64_t)pb.N, (uint64_t)pb.K / 2, BK / 2, BM,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
   if (e != cudaSuccess) return e;
+  // A tile's scales (128 rows x srow bytes, contiguous) come by one bulk
+  // copy when they fit the buffer, there are at least two stages per tile
+  // (so both decode groups take part in every tile) and every copy stays
+  // 16-byte aligned: rows start at multiples of 128, so N * srow and the
+  // array's address must be multiples of 16.
+  const int srow = (f == Fmt::NF4) ? (int)(pb.K / 64) * 4 : (int)(pb.K / 32);
+  const int tile_scales = (pb.K / BK >= 2) && (BM * srow <= kScaleBuf) &&
+                          ((pb.N * srow) % 16 == 0) &&
+                          (reinterpret_cast<uintptr_t>(pb.scale) % 16 == 0);
   const size_t smem = gemm_smem_bytes(pb.E);
   auto k = (f == Fmt::NF4) ? gemm_kernel<Fmt::NF4> : gemm_kernel<Fmt::MXFP4>;
   e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<num_sms, kThreads, smem, s>>>(pb, tmx, tmw);
+  k<<<num_sms, kThreads, smem, s>>>(pb, tmx, tmx32, tmw, srow, tile_scales);
   return cudaGetLastError();
 }
 
