@@ -177,18 +177,6 @@ gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
     }
     xkey = (int64_t)tok * npass + pass;
   };
-  // pair table: entry b -> bf16 (value of the even element, value of the odd
-  // element) in every lane's column; 16-byte stores fill four columns.  It
-  // touches no caller memory, so it runs before the dependency wait.
-  for (int i = threadIdx.x; i < 256 * 8; i += kThreads) {
-    const uint32_t b = (uint32_t)i >> 3;
-    const uint32_t qe = (F == Fmt::NF4) ? (b >> 4) : (b & 15u);
-    const uint32_t qo = (F == Fmt::NF4) ? (b & 15u) : (b >> 4);
-    const uint32_t v =
-        (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qe))) |
-        ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qo))) << 16);
-    *reinterpret_cast<uint4*>(base + lay.lut + b * 256 + (i & 7) * 16) = make_uint4(v, v, v, v);
-  }
   // Programmatic dependent launch.  x may be written by the kernel launched
   // just before this one, so it is read only after grid_dependency_wait;
   // with GBW_FLAG_OVERLAP_PREV the offsets, row map, codes and scales are
@@ -204,9 +192,27 @@ gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
     }
   };
   if (!early) ready();
-  // independent global loads first: the offsets and the first row's token
+  // independent global loads first (the offsets and the first row's token),
+  // so the table below is built while they are in flight
   const OffsetRegs offr = prefetch_offsets(pb.offsets, pb.E);
   int32_t tok = g0 < g1 ? token_of_row(pb.row_to_token, p, pb.T, pb.err) : 0;
+  // pair table: entry b -> bf16 (value of the even element, value of the odd
+  // element) in every lane's column.  Thread b < 256 builds entry b and
+  // writes its 128-byte row with eight 16-byte stores, starting at chunk
+  // b % 8 so the 32 stores of a warp instruction spread over all banks.
+  // It touches no caller memory.
+  if (threadIdx.x < 256) {
+    const uint32_t b = threadIdx.x;
+    const uint32_t qe = (F == Fmt::NF4) ? (b >> 4) : (b & 15u);
+    const uint32_t qo = (F == Fmt::NF4) ? (b & 15u) : (b >> 4);
+    const uint32_t v =
+        (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qe))) |
+        ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qo))) << 16);
+    uint8_t* row = base + lay.lut + b * 256;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<uint4*>(row + ((c + b) & 7u) * 16) = make_uint4(v, v, v, v);
+  }
   if (!early && g0 < g1) load_x(tok, 0);
   commit_offsets(offr, pb.offsets, pb.E, pb.P, off_s, pb.err);  // barrier inside
 
