@@ -7,9 +7,13 @@
 // in HBM.
 //
 // B200 design (one persistent CTA per SM, 16 warps):
-//   tile  = 128 weight rows (MMA M) x up to 256 routed rows (MMA N) x K: the
-//           matmul runs as out^T = W x^T ("swap AB"), so an expert with few
-//           routed rows gets a narrow MMA N instead of a padded M;
+//   tile  = 128 weight rows (MMA M) x up to 512 routed rows x K: the matmul
+//           runs as out^T = W x^T ("swap AB"), so an expert with few routed
+//           rows gets a narrow MMA N instead of a padded M.  Rows past 256
+//           go to the second accumulator half, fed by the same decoded A
+//           stage, so a large expert's weights are decoded half as often
+//           (wide tiles: identity rows only; gathered rows keep 256-row
+//           tiles, whose cp.async gather cannot feed 64 KB stages);
 //   warps 4-11  decode, two groups of four warps taking alternate 64-K
 //               stages.  A stage's packed bytes (128 rows x 32 bytes) arrive
 //               by TMA into the group's 2-slot ring; a tile's scales (128
@@ -20,20 +24,22 @@
 //               the 128B-swizzled, K-major A tile (one slot per group).
 //               These warps bound the kernel by the instructions they issue,
 //               so their loop does no per-stage divisions or global loads;
-//   warp 2      activations, identity rows: one 2-D TMA tile (64 K x 256
-//               rows, 128B swizzle) per stage into a 4-stage ring (32-row
-//               boxes for a partial tile);
+//   warp 2      activations, identity rows: 2-D TMA boxes (64 K x 256 rows,
+//               128B swizzle; 32-row boxes for a partial half) into a
+//               2-stage ring of 64 KB stages;
 //   warps 0,2,3 activations gathered through row_to_token: eight consecutive
 //               lanes copy one row's 128 bytes of a stage with 16-byte
-//               cp.async, so each warp instruction moves four whole rows;
+//               cp.async, so each warp instruction moves four whole rows
+//               (4-stage ring of 32 KB stages);
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (A and B from
 //               shared memory, fp32 accumulator in TMEM) and tcgen05.commit;
 //   warps 12-15 epilogue: tcgen05.ld 32 accumulator columns (routed rows) of
 //               the warp's 32 weight rows, round to bf16, transpose 32 x 32
 //               through shared memory and write whole 64-byte row segments.
-// Tensor memory holds two 128 x 256 fp32 accumulators, so the epilogue of one
-// tile overlaps the mainloop of the next.
-// Scheduler: tiles (expert, 128-row weight tile, 256-row token tile) with
+// Tensor memory holds two 128 x 256 fp32 accumulator halves: tiles of up to
+// 256 rows alternate between them, so the epilogue of one overlaps the
+// mainloop of the next; a wider tile takes both.
+// Scheduler: tiles (expert, 128-row weight tile, token tile) with
 // zero-row experts skipped, enumerated from expert_offsets by every CTA and
 // dealt round-robin (token tiles innermost, so CTAs running at the same time
 // share one weight tile through L2).
@@ -44,9 +50,10 @@ namespace gbw {
 namespace {
 
 constexpr int BM = 128;   // weight rows per tile (MMA M)
-constexpr int BT = 256;   // routed rows per tile (max MMA N)
+constexpr int BH = 256;   // routed rows per accumulator half (max MMA N)
 constexpr int BK = 64;    // K per stage
-constexpr int XS = 4;     // activation ring stages
+constexpr int kXRingBytes = 128 * 1024;  // activation ring, either tile shape
+constexpr int kXSMax = 4;                // most activation stages (barriers)
 constexpr int AS = 2;     // decoded-weight (A operand) ring stages: one per decode group
 static_assert(AS % 2 == 0, "the two decode groups own alternate A slots");
 constexpr int WG = 2;     // packed-weight ring stages per decode group
@@ -54,7 +61,20 @@ constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 static_assert(BK == 64, "the MMA issuer unrolls four K = 16 steps per stage");
 
-constexpr int kXStageBytes = BT * BK * 2;      // 32 KB
+constexpr int kXHalfBytes = BH * BK * 2;       // 32 KB
+
+// Tile shapes.  Wide (identity rows, activations by TMA): up to 512 routed
+// rows, both accumulator halves fed by one decoded A stage, so a large
+// expert's weights are decoded half as often; two 64 KB activation stages.
+// Narrow (gathered rows): up to 256 routed rows, four 32 KB stages -- the
+// cp.async gather cannot keep two 64 KB stages fed.
+template <bool W>
+struct TileCfg {
+  static constexpr int BT = W ? 512 : 256;
+  static constexpr int XS = W ? 2 : 4;
+  static constexpr int kXStageBytes = BT * BK * 2;
+  static_assert(XS * kXStageBytes == kXRingBytes && XS <= kXSMax, "ring");
+};
 constexpr int kAStageBytes = BM * BK * 2;      // 16 KB
 constexpr int kWStageBytes = BM * BK / 2;      // 4 KB: 128 rows x 32 packed bytes
 constexpr int kScaleBuf = 16 * 1024;           // one tile's scales (double buffered)
@@ -65,14 +85,35 @@ constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
 struct Smem {
   // byte offsets inside the dynamic shared memory block (1024-aligned base)
   static constexpr int x = 0;
-  static constexpr int a = x + XS * kXStageBytes;
+  static constexpr int a = x + kXRingBytes;
   static constexpr int w = a + AS * kAStageBytes;    // packed weights, 2 groups
   static constexpr int sc = w + 2 * WG * kWStageBytes;   // tile scales, 2 buffers
   static constexpr int epi = sc + 2 * kScaleBuf;         // epilogue transpose
   static constexpr int bars = epi + 4 * kEpiWarpBytes;
-  static constexpr int nbars = 2 * XS + 2 * AS + 4 * WG + 4 + 5;
+  static constexpr int nbars = 2 * kXSMax + 2 * AS + 4 * WG + 4 + 5;
   static constexpr int misc = bars + nbars * 8;      // tmem base, abort flag
   static constexpr int tables = misc + 16;           // offsets[E+1], tile_start[E+1]
+};
+
+// Which accumulator half (256 TMEM columns) a tile uses.  A tile of up to
+// 256 rows takes the next half and the halves alternate, so its epilogue
+// overlaps the next tile's mainloop; a wider tile takes both halves (the
+// next one first).  The MMA thread and the epilogue warps step identical
+// copies, so they agree on halves and on each half's barrier phase.
+struct AccSched {
+  uint32_t h = 0;              // next half
+  uint32_t use0 = 0, use1 = 0;  // tiles that have used each half so far
+  // parity of the current use of half k (registers, no indexed array)
+  __device__ __forceinline__ uint32_t phase(uint32_t k) const { return (k ? use1 : use0) & 1u; }
+  __device__ __forceinline__ void next(bool wide) {
+    if (wide) {
+      ++use0;
+      ++use1;
+    } else {
+      if (h) ++use1; else ++use0;
+      h ^= 1u;
+    }
+  }
 };
 
 struct TileInfo {
@@ -80,7 +121,7 @@ struct TileInfo {
 };
 
 __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
-                                              const int32_t* ts, int32_t E) {
+                                              const int32_t* ts, int32_t E, int32_t BT) {
   int32_t lo = 0, hi = E - 1;  // last e with ts[e] <= t
   while (lo < hi) {
     int32_t mid = (lo + hi + 1) >> 1;
@@ -98,12 +139,15 @@ __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
   return ti;
 }
 
-template <Fmt F>
+template <Fmt F, bool W>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
             const __grid_constant__ CUtensorMap tmx32,
             const __grid_constant__ CUtensorMap tmw, const int srow,
             const int tile_scales) {
+  constexpr int BT = TileCfg<W>::BT;  // routed rows per tile
+  constexpr int XS = TileCfg<W>::XS;  // activation ring stages
+  constexpr int kXStageBytes = TileCfg<W>::kXStageBytes;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128B-swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -172,20 +216,25 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       // a partial tile)
       if (warp == 2 && lane == 0) {
         for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-          const TileInfo ti = tile_info(t, off_s, ts_s, E);
+          const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
           for (int kb = 0; kb < NK; ++kb, ++g) {
             const uint32_t s = g % XS, ph = (g / XS) & 1u;
             if (!(ok = mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err))) break;
             uint8_t* dst = smem + Smem::x + s * kXStageBytes;
-            if (ti.nv == BT) {
-              mbar_arrive_expect_tx(&x_full[s], kXStageBytes);
-              tma_load_2d(dst, &tmx, kb * BK, ti.p0, &x_full[s]);
-            } else {
-              const int nb = (ti.nv + 31) >> 5;  // 32-row boxes of 4 KB
-              mbar_arrive_expect_tx(&x_full[s], (uint32_t)nb * (32 * BK * 2));
-              for (int b = 0; b < nb; ++b)
-                tma_load_2d(dst + b * (32 * BK * 2), &tmx32, kb * BK, ti.p0 + 32 * b, &x_full[s]);
-            }
+            // each half: one 256-row box when full, else the 32-row boxes it uses
+            const int n0 = min(ti.nv, BH), n1 = ti.nv - n0;
+            const int b0 = n0 == BH ? 0 : (n0 + 31) >> 5;
+            const int b1 = n1 == BH ? 0 : (n1 + 31) >> 5;
+            const uint32_t bytes = (n0 == BH ? kXHalfBytes : b0 * (32 * BK * 2)) +
+                                   (n1 == BH ? kXHalfBytes : b1 * (32 * BK * 2));
+            mbar_arrive_expect_tx(&x_full[s], bytes);
+            if (n0 == BH) tma_load_2d(dst, &tmx, kb * BK, ti.p0, &x_full[s]);
+            for (int b = 0; b < b0; ++b)
+              tma_load_2d(dst + b * (32 * BK * 2), &tmx32, kb * BK, ti.p0 + 32 * b, &x_full[s]);
+            if (n1 == BH) tma_load_2d(dst + kXHalfBytes, &tmx, kb * BK, ti.p0 + BH, &x_full[s]);
+            for (int b = 0; b < b1; ++b)
+              tma_load_2d(dst + kXHalfBytes + b * (32 * BK * 2), &tmx32, kb * BK,
+                          ti.p0 + BH + 32 * b, &x_full[s]);
           }
         }
         if (*abort)
@@ -208,7 +257,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       const int chunk = lane & 7;
       const int r0 = 4 * gw + (lane >> 3);
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tile_info(t, off_s, ts_s, E);
+        const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
         int32_t tk[kRows];
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
@@ -239,18 +288,21 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     // their issue time (measured: a 128 x 256 x 16 MMA takes 128 cycles when
     // issued back to back, ~240 with descriptors rebuilt around it).
     if (lane == 0) {
-      uint32_t g = 0, it = 0;
+      uint32_t g = 0;
       bool ok = true;
       const uint64_t xdesc0 = make_sdesc_sw128(smem_u32(smem + Smem::x), 16, 1024);
       const uint64_t adesc0 = make_sdesc_sw128(smem_u32(smem + Smem::a), 16, 1024);
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
-        const TileInfo ti = tile_info(t, off_s, ts_s, E);
-        const uint32_t nmma = (uint32_t)((ti.nv + 15) & ~15);
-        const uint32_t idesc = make_idesc_bf16(BM, nmma, 0, 0);
-        const uint32_t ab = it & 1u;
-        if (!(ok = mbar_wait(&acc_empty[ab], ((it >> 1) & 1u) ^ 1u, abort, pb.err))) break;
+      AccSched acc;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
+        const bool wide = ti.nv > BH;
+        const uint32_t h0 = acc.h, h1 = acc.h ^ 1u;
+        const uint32_t idesc0 = make_idesc_bf16(BM, wide ? (uint32_t)BH : (uint32_t)((ti.nv + 15) & ~15), 0, 0);
+        const uint32_t idesc1 = make_idesc_bf16(BM, (uint32_t)((ti.nv - BH + 15) & ~15), 0, 0);
+        if (!(ok = mbar_wait(&acc_empty[h0], acc.phase(h0) ^ 1u, abort, pb.err))) break;
+        if (wide && !(ok = mbar_wait(&acc_empty[h1], acc.phase(h1) ^ 1u, abort, pb.err))) break;
         tc_fence_after();
-        const uint32_t dacc = tmem + ab * 256u;
+        const uint32_t d0 = tmem + h0 * 256u, d1 = tmem + h1 * 256u;
         for (int kb = 0; kb < NK; ++kb, ++g) {
           const uint32_t xs = g % XS, as = g % AS;
           if (!(ok = mbar_wait(&a_full[as], (g / AS) & 1u, abort, pb.err))) break;
@@ -259,14 +311,25 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
           tc_fence_after();
           const uint64_t ad = adesc0 + (uint64_t)((as * kAStageBytes) >> 4);
           const uint64_t bd = xdesc0 + (uint64_t)((xs * kXStageBytes) >> 4);
-          tc_mma_ss(dacc, ad, bd, idesc, kb != 0);
-          tc_mma_ss(dacc, ad + 2, bd + 2, idesc, 1u);  // +32 bytes: next 16 K
-          tc_mma_ss(dacc, ad + 4, bd + 4, idesc, 1u);
-          tc_mma_ss(dacc, ad + 6, bd + 6, idesc, 1u);
+          // one decoded A stage feeds both halves of a wide tile
+          tc_mma_ss(d0, ad, bd, idesc0, kb != 0);
+          tc_mma_ss(d0, ad + 2, bd + 2, idesc0, 1u);  // +32 bytes: next 16 K
+          tc_mma_ss(d0, ad + 4, bd + 4, idesc0, 1u);
+          tc_mma_ss(d0, ad + 6, bd + 6, idesc0, 1u);
+          if (wide) {
+            const uint64_t bd1 = bd + (uint64_t)(kXHalfBytes >> 4);
+            tc_mma_ss(d1, ad, bd1, idesc1, kb != 0);
+            tc_mma_ss(d1, ad + 2, bd1 + 2, idesc1, 1u);
+            tc_mma_ss(d1, ad + 4, bd1 + 4, idesc1, 1u);
+            tc_mma_ss(d1, ad + 6, bd1 + 6, idesc1, 1u);
+          }
           tc_commit(&x_empty[xs]);
           tc_commit(&a_empty[as]);
         }
-        if (ok) tc_commit(&acc_full[ab]);
+        if (!ok) break;
+        tc_commit(&acc_full[h0]);
+        if (wide) tc_commit(&acc_full[h1]);
+        acc.next(wide);
       }
       // every MMA this thread issued has finished before TMEM is released
       tc_commit(mma_done);
@@ -301,11 +364,11 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     const uint32_t nh = total > grp ? (total - grp + 1) / 2 : 0;  // this group's stages
     // first weight row (e * N + n0) of local tile tl
     auto tile_row = [&](int64_t tl) -> int64_t {
-      const TileInfo ti = tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E);
+      const TileInfo ti = tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E, BT);
       return (int64_t)ti.e * N + ti.n0;
     };
     auto tile_n0 = [&](int64_t tl) -> int32_t {
-      return tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E).n0;
+      return tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E, BT).n0;
     };
     // cursor: local tile tl and stage kb of group stage h; step() = h + 1
     struct Cursor {
@@ -480,47 +543,55 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     // Thread t of warp q holds output column n0 + 32q + t for 32 routed rows
     // per TMEM chunk; a 32 x 32 bf16 transpose through shared memory turns
     // that into 64 contiguous bytes of one output row per thread, written
-    // with four 16-byte stores.
+    // with four 16-byte stores.  A wide tile's halves are drained in order,
+    // each released as soon as it has been read.
     const uint32_t q = (uint32_t)warp & 3u;
     uint8_t* stage = smem + Smem::epi + q * kEpiWarpBytes;
-    uint32_t it = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-      const TileInfo ti = tile_info(t, off_s, ts_s, E);
-      const uint32_t ab = it & 1u;
-      const uint32_t tlane = tmem + ((q * 32u) << 16) + ab * 256u;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (it >> 1) & 1u, abort, pb.err));
-      if (!ok) break;
-      tc_fence_after();
-      const int nchunks = (ti.nv + 31) >> 5;
+    AccSched acc;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
+      const bool wide = ti.nv > BH;
       const int ncol0 = ti.n0 + (int)q * 32;  // first output column of this warp
-      for (int c = 0; c < nchunks; ++c) {
-        uint32_t r[32];
-        tmem_load_32x32b_x32(tlane + c * 32, r);
-        if (c == nchunks - 1) {
-          tc_fence_before();
+      const int sub = lane & 3;               // 16-byte piece of a row
+      const bool subok = ncol0 + sub * 8 < N;
+      for (int part = 0; part < (wide ? 2 : 1) && ok; ++part) {
+        const uint32_t hf = part ? acc.h ^ 1u : acc.h;
+        const int row0 = part * BH;
+        const int rows = part ? ti.nv - BH : min(ti.nv, BH);
+        ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[hf], acc.phase(hf), abort, pb.err));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tlane = tmem + ((q * 32u) << 16) + hf * 256u;
+        const int nchunks = (rows + 31) >> 5;
+        for (int c = 0; c < nchunks; ++c) {
+          uint32_t r[32];
+          tmem_load_32x32b_x32(tlane + c * 32, r);
+          if (c == nchunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[hf]);
+          }
+          // thread = output column ncol0 + lane, r[j] = routed row c*32 + j
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            *reinterpret_cast<uint16_t*>(stage + j * kEpiRowBytes + lane * 2) =
+                __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[j])));
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        }
-        // thread = output column ncol0 + lane, r[j] = routed row c*32 + j
+          // four lanes write one routed row's 64 bytes, so each store
+          // instruction covers eight whole row segments (full 32-byte sectors)
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          *reinterpret_cast<uint16_t*>(stage + j * kEpiRowBytes + lane * 2) =
-              __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[j])));
-        __syncwarp();
-        // four lanes write one routed row's 64 bytes, so each store
-        // instruction covers eight whole row segments (full 32-byte sectors)
-        const int sub = lane & 3;              // 16-byte piece of the row
-        const bool subok = ncol0 + sub * 8 < N;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int rr = (lane >> 2) + 8 * v;  // row within the chunk
-          const int row = c * 32 + rr;         // routed row within the tile
-          if (row < ti.nv && subok)
-            *reinterpret_cast<uint4*>(pb.out + (int64_t)(ti.p0 + row) * N + ncol0 + sub * 8) =
-                *reinterpret_cast<const uint4*>(stage + rr * kEpiRowBytes + sub * 16);
+          for (int v = 0; v < 4; ++v) {
+            const int rr = (lane >> 2) + 8 * v;  // row within the chunk
+            const int row = c * 32 + rr;         // routed row within the half
+            if (row < rows && subok)
+              *reinterpret_cast<uint4*>(pb.out + (int64_t)(ti.p0 + row0 + row) * N + ncol0 + sub * 8) =
+                  *reinterpret_cast<const uint4*>(stage + rr * kEpiRowBytes + sub * 16);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
+      acc.next(wide);
     }
   }
 
@@ -581,11 +652,11 @@ cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
                         cudaStream_t s) {
   if (pb.P == 0 || pb.N == 0) return cudaSuccess;
   CUtensorMap tmx;
-  // identity rows: tiles of 64 K x 256 rows; gathered rows use cp.async and
+  // identity rows: boxes of 64 K x 256 rows (one per tile half); gathered rows use cp.async and
   // never read this map
   cudaError_t e = make_map_2d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pb.x,
                               (uint64_t)pb.K, (uint64_t)(pb.T > 0 ? pb.T : 1),
-                              (uint64_t)pb.K * 2, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B);
+                              (uint64_t)pb.K * 2, BK, BH, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   CUtensorMap tmx32;  // the same rows in boxes of 32, for partial tiles
   e = make_map_2d(&tmx32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pb.x,
@@ -609,7 +680,11 @@ cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
                           ((pb.N * srow) % 16 == 0) &&
                           (reinterpret_cast<uintptr_t>(pb.scale) % 16 == 0);
   const size_t smem = gemm_smem_bytes(pb.E);
-  auto k = (f == Fmt::NF4) ? gemm_kernel<Fmt::NF4> : gemm_kernel<Fmt::MXFP4>;
+  // wide tiles when activations come by TMA (identity rows), narrow when
+  // they are gathered through row_to_token
+  const bool wide = pb.row_to_token == nullptr;
+  auto k = (f == Fmt::NF4) ? (wide ? gemm_kernel<Fmt::NF4, true> : gemm_kernel<Fmt::NF4, false>)
+                           : (wide ? gemm_kernel<Fmt::MXFP4, true> : gemm_kernel<Fmt::MXFP4, false>);
   e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
