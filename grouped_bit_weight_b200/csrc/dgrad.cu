@@ -9,19 +9,22 @@
 // transposed orientation.
 //
 // B200 design (one persistent CTA per SM, 16 warps):
-//   tile = 128 routed rows (MMA M) x 256 output columns k (MMA N), reduced
-//          over N in stages of 64 weight rows;
-//   warp 0      TMA: dy tile [128 x 64] (128B swizzle, K-major A operand)
+//   tile = up to 256 routed rows x 256 output columns k (MMA N), reduced
+//          over N in stages of 64 weight rows; the routed rows go 128 at a
+//          time (MMA M) to the two TMEM accumulator halves, both fed by one
+//          decoded B stage, so a weight slab is decoded once per 256 rows;
+//   warp 0      TMA: dy tile [256 x 64] (128B swizzle, K-major A operand)
 //               and the packed slab [64 weight rows x 128 bytes] (swizzled so
-//               the decode reads are bank-conflict free) -> smem ring (4)
+//               the decode reads are bank-conflict free) -> smem ring (3)
 //   warps 4-11  decode: thread (weight row n, 64-wide k block j) decodes 64
 //               weights with the register table and stores them as one
 //               128-byte row of the MN-major, 128B-swizzled B operand
 //               (3-stage ring); the decoded tile lives only in smem
 //   warp 1      tcgen05.mma (A and B from smem, fp32 accumulator in TMEM)
-//   warps 12-15 epilogue: tcgen05.ld -> bf16 -> 16-byte stores of dx rows;
-//               two TMEM accumulators (2 x 256 columns) let the epilogue of
-//               one tile overlap the mainloop of the next.
+//   warps 12-15 epilogue: tcgen05.ld -> bf16 -> 16-byte stores of dx rows.
+//               Tiles of up to 128 rows alternate between the two TMEM
+//               accumulator halves (2 x 256 columns), so the epilogue of one
+//               overlaps the mainloop of the next; a wider tile takes both.
 // Tiles (expert, k tile, routed-row tile) with routed-row tiles innermost, so
 // CTAs running together share one packed weight slab through L2.
 #include "common.cuh"
@@ -30,16 +33,18 @@
 namespace gbw {
 namespace {
 
-constexpr int BM = 128;   // routed rows per tile (MMA M)
+constexpr int BM = 128;   // routed rows per accumulator half (MMA M)
+constexpr int BMW = 256;  // routed rows per tile: two halves share each decoded B
 constexpr int BN = 256;   // output k columns per tile (MMA N)
 constexpr int BR = 64;    // weight rows (reduction) per stage
-constexpr int LS = 4;     // load ring stages (dy + packed)
+constexpr int LS = 3;     // load ring stages (dy + packed)
 constexpr int DS = 3;     // decoded-B ring stages
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
 static_assert(BR == 64, "the MMA issuer unrolls four 16-row steps per stage");
 
-constexpr int kAStageBytes = BM * BR * 2;   // 16 KB
+constexpr int kAStageBytes = BMW * BR * 2;  // 32 KB
+constexpr int kAHalfBytes = BM * BR * 2;    // 16 KB
 constexpr int kWStageBytes = BR * BN / 2;   // 8 KB
 constexpr int kLStageBytes = kAStageBytes + kWStageBytes;
 constexpr int kBStageBytes = BR * BN * 2;   // 32 KB
@@ -65,16 +70,36 @@ __device__ __forceinline__ DTile dtile_info(int64_t t, const int32_t* off,
     if (ts[mid] <= t) lo = mid; else hi = mid - 1;
   }
   const int32_t cnt = off[lo + 1] - off[lo];
-  const int32_t mt_n = (cnt + BM - 1) / BM;
+  const int32_t mt_n = (cnt + BMW - 1) / BMW;
   const int32_t u = (int32_t)(t - ts[lo]);
   const int32_t kt = u / mt_n, mt = u - kt * mt_n;
   DTile d;
   d.e = lo;
   d.k0 = kt * BN;
-  d.p0 = off[lo] + mt * BM;
-  d.nv = min(BM, cnt - mt * BM);
+  d.p0 = off[lo] + mt * BMW;
+  d.nv = min(BMW, cnt - mt * BMW);
   return d;
 }
+
+// Which accumulator half (256 TMEM columns) a tile uses: a tile of up to
+// 128 routed rows takes the next half and the halves alternate, so its
+// epilogue overlaps the next tile's mainloop; a wider tile takes both (the
+// next one first).  The MMA thread and the epilogue warps step identical
+// copies, so they agree on halves and on each half's barrier phase.
+struct AccSched {
+  uint32_t h = 0;
+  uint32_t use0 = 0, use1 = 0;
+  __device__ __forceinline__ uint32_t phase(uint32_t k) const { return (k ? use1 : use0) & 1u; }
+  __device__ __forceinline__ void next(bool wide) {
+    if (wide) {
+      ++use0;
+      ++use1;
+    } else {
+      if (h) ++use1; else ++use0;
+      h ^= 1u;
+    }
+  }
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
 dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
@@ -119,7 +144,7 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
     tma_prefetch_desc(&tmw);
   }
   load_offsets_clamped(pb.offsets, E, pb.P, off_s, pb.err);
-  tile_prefix(off_s, E, BM, nkt, ts_s);
+  tile_prefix(off_s, E, BMW, nkt, ts_s);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -150,20 +175,23 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      uint32_t g = 0, it = 0;
+      uint32_t g = 0;
       bool ok = true;
       // descriptors advance by 64-bit adds (start address in 16-byte units):
       // nothing but the MMAs runs between them in this thread
       const uint64_t adesc0 = make_sdesc_sw128(smem_u32(smem + Smem::ld), 16, 1024);
       const uint64_t bdesc0 = make_sdesc_sw128(smem_u32(smem + Smem::b), 1024, 4096);
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+      AccSched acc;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const DTile d = dtile_info(t, off_s, ts_s, E);
+        const bool wide = d.nv > BM;
         const uint32_t nmma = (uint32_t)min((int64_t)BN, K - d.k0);
         const uint32_t idesc = make_idesc_bf16(BM, nmma, 0, 1);
-        const uint32_t ab = it & 1u;
-        if (!(ok = mbar_wait(&acc_empty[ab], ((it >> 1) & 1u) ^ 1u, abort, pb.err))) break;
+        const uint32_t h0 = acc.h, h1 = acc.h ^ 1u;
+        if (!(ok = mbar_wait(&acc_empty[h0], acc.phase(h0) ^ 1u, abort, pb.err))) break;
+        if (wide && !(ok = mbar_wait(&acc_empty[h1], acc.phase(h1) ^ 1u, abort, pb.err))) break;
         tc_fence_after();
-        const uint32_t dacc = tmem + ab * 256u;
+        const uint32_t d0 = tmem + h0 * 256u, d1 = tmem + h1 * 256u;
         for (int ks = 0; ks < NS; ++ks, ++g) {
           const uint32_t ls = g % LS, bs = g % DS;
           if (!(ok = mbar_wait(&ld_full[ls], (g / LS) & 1u, abort, pb.err))) break;
@@ -171,14 +199,25 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
           tc_fence_after();
           const uint64_t ad = adesc0 + (uint64_t)((ls * kLStageBytes) >> 4);
           const uint64_t bd = bdesc0 + (uint64_t)((bs * kBStageBytes) >> 4);
-          tc_mma_ss(dacc, ad, bd, idesc, ks != 0);
-          tc_mma_ss(dacc, ad + 2, bd + 512, idesc, 1u);   // A +32 B, B +8 KB: next 16 n
-          tc_mma_ss(dacc, ad + 4, bd + 1024, idesc, 1u);
-          tc_mma_ss(dacc, ad + 6, bd + 1536, idesc, 1u);
+          // one decoded B stage feeds both halves of a wide tile
+          tc_mma_ss(d0, ad, bd, idesc, ks != 0);
+          tc_mma_ss(d0, ad + 2, bd + 512, idesc, 1u);   // A +32 B, B +8 KB: next 16 n
+          tc_mma_ss(d0, ad + 4, bd + 1024, idesc, 1u);
+          tc_mma_ss(d0, ad + 6, bd + 1536, idesc, 1u);
+          if (wide) {
+            const uint64_t ad1 = ad + (uint64_t)(kAHalfBytes >> 4);  // dy rows 128..255
+            tc_mma_ss(d1, ad1, bd, idesc, ks != 0);
+            tc_mma_ss(d1, ad1 + 2, bd + 512, idesc, 1u);
+            tc_mma_ss(d1, ad1 + 4, bd + 1024, idesc, 1u);
+            tc_mma_ss(d1, ad1 + 6, bd + 1536, idesc, 1u);
+          }
           tc_commit(&ld_empty[ls]);
           tc_commit(&b_empty[bs]);
         }
-        if (ok) tc_commit(&acc_full[ab]);
+        if (!ok) break;
+        tc_commit(&acc_full[h0]);
+        if (wide) tc_commit(&acc_full[h1]);
+        acc.next(wide);
       }
       tc_commit(mma_done);
       mbar_drain(mma_done, 0);
@@ -254,17 +293,20 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
   } else if (warp >= 12) {
     // ---------------- epilogue ----------------
     const uint32_t q = (uint32_t)warp & 3u;
-    const int m = (int)(q * 32 + lane);
-    uint32_t it = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    AccSched acc;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
       const DTile d = dtile_info(t, off_s, ts_s, E);
-      const uint32_t ab = it & 1u;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (it >> 1) & 1u, abort, pb.err));
+      const bool wide = d.nv > BM;
+      for (int part = 0; part < (wide ? 2 : 1); ++part) {
+      const uint32_t hf = part ? acc.h ^ 1u : acc.h;
+      const int m = part * BM + (int)(q * 32 + lane);  // routed row in the tile
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[hf], acc.phase(hf), abort, pb.err));
       if (!ok) break;
       tc_fence_after();
       const int width = (int)min((int64_t)BN, K - d.k0);
       const int nchunks = width >> 5;
-      const uint32_t taddr = tmem + ((q * 32u) << 16) + ab * 256u;
+      const uint32_t taddr = tmem + ((q * 32u) << 16) + hf * 256u;
       uint16_t* dst = pb.out + (int64_t)(d.p0 + m) * K + d.k0;
       for (int c = 0; c < nchunks; ++c) {
         uint32_t r[32];
@@ -272,7 +314,7 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
         if (c == nchunks - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          if (lane == 0) mbar_arrive(&acc_empty[hf]);
         }
         if (m < d.nv) {
 #pragma unroll
@@ -286,6 +328,8 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
           }
         }
       }
+      }
+      acc.next(wide);
     }
   }
 
@@ -303,16 +347,18 @@ cudaError_t make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
 cudaError_t launch_dgrad(const GroupedProblem& pb, int num_sms, cudaStream_t s) {
   if (pb.P == 0 || pb.K == 0) return cudaSuccess;
   CUtensorMap tma, tmw;
-  // dy [P, N] bf16: box 64 (reduction) x 128 rows, 128B swizzle
+  // dy [P, N] bf16: box 64 (reduction) x 256 rows, 128B swizzle
   cudaError_t e = make_map_2d(&tma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pb.x,
                               (uint64_t)pb.N, (uint64_t)pb.P, (uint64_t)pb.N * 2,
-                              BR, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+                              BR, BMW, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   // packed [E*N, K/2] u8: box 128 bytes x 64 rows, 128B swizzle
   e = make_map_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.w, (uint64_t)pb.K / 2,
                   (uint64_t)pb.E * (uint64_t)pb.N, (uint64_t)pb.K / 2, BN / 2, BR,
                   CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
+  static_assert(1024 + Smem::tables + 8 * (1024 + 1) <= 232448,
+                "shared memory for 1024 experts exceeds the 227 KB a CTA can have");
   const size_t smem = 1024 + Smem::tables + sizeof(int32_t) * 2 * (size_t)(pb.E + 1);
   e = cudaFuncSetAttribute(dgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
