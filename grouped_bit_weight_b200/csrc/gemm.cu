@@ -210,10 +210,9 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     uint32_t g = 0;
     bool ok = true;
     if (!gathered) {
-      // routed row p reads x row p: one 2-D TMA tile (64 K x 256 rows) per
-      // stage; a tile with fewer rows loads only the 32-row boxes it uses
-      // (activation reads from L2 bound the kernel, and most experts end in
-      // a partial tile)
+      // routed row p reads x row p: per stage, each 256-row half of the
+      // tile is one 2-D TMA box (64 K x 256 rows), or only the 32-row boxes
+      // a partial half uses (most experts end in a partial tile)
       if (warp == 2 && lane == 0) {
         for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
           const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
