@@ -590,7 +590,7 @@ def cpu_baseline():
     nbytes = gemv_bytes("nf4", 8, GU.N, GU.K, 1) + gemv_bytes("nf4", 8, DN.N, DN.K, 8)
     step()
     n, t = 0, time.perf_counter()
-    while time.perf_counter() - t < 10.0 and n < 200:
+    while time.perf_counter() - t < 10.0 and n < 20000:
         step()
         n += 1
     dt = time.perf_counter() - t
