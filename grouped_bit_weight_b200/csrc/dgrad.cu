@@ -230,38 +230,46 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
     const int rr = n & 7;                       // row inside the 8-row atom
     const int64_t my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const uint32_t total = (uint32_t)(my_tiles * NS);
-    // absmax of stage g for (row n, block j), fetched three stages ahead
-    int64_t pf_tile = -1;
-    int32_t pf_e = 0, pf_k0 = 0;
-    auto scale_at = [&](uint32_t g) -> float {
-      if (g >= total) return 0.0f;
-      const int64_t ti_idx = g / NS;
-      if (ti_idx != pf_tile) {
-        pf_tile = ti_idx;
-        const DTile d = dtile_info(blockIdx.x + ti_idx * gridDim.x, off_s, ts_s, E);
-        pf_e = d.e;
-        pf_k0 = d.k0;
-      }
-      if (pf_k0 + 64 * j >= K) return 0.0f;
-      const int64_t wrow = (int64_t)pf_e * N + (int64_t)(g % NS) * BR + n;
-      return __ldg(reinterpret_cast<const float*>(pb.scale) + wrow * (K / 64) + pf_k0 / 64 + j);
+    // These warps bound the kernel by the instructions they issue, so the
+    // bookkeeping is incremental: a cursor (local tile, stage) per
+    // look-ahead distance steps one stage at a time and looks a tile up only
+    // when it enters a new one (no divisions by the stage count), and the
+    // absmax of stage g + 4 is loaded into the slot stage g has just used
+    // (fixed slots: a queue rotated by register copies would wait on each
+    // load one stage after issuing it).
+    struct Cursor {
+      int64_t tl;
+      int ks;
     };
-    float s0 = scale_at(0), s1 = scale_at(1), s2 = scale_at(2);
-    int64_t cur_tile = -1;
-    bool jvalid = false;
-    for (uint32_t g = 0; g < total; ++g) {
-      const float a = s0;
-      s0 = s1;
-      s1 = s2;
-      s2 = scale_at(g + 3);
-      const int64_t ti_idx = g / NS;
-      if (ti_idx != cur_tile) {
-        cur_tile = ti_idx;
-        const DTile d = dtile_info(blockIdx.x + ti_idx * gridDim.x, off_s, ts_s, E);
-        jvalid = d.k0 + 64 * j < K;
+    // absmax cursor: the scale row of (weight row n, block j) in its tile
+    Cursor sc_cur{0, 0};
+    const float* srow = nullptr;  // absmax of weight row (e*N + n) at block k0/64 + j, or null
+    auto srow_of = [&](int64_t tl) -> const float* {
+      const DTile d = dtile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E);
+      if (d.k0 + 64 * j >= K) return nullptr;
+      return reinterpret_cast<const float*>(pb.scale) + ((int64_t)d.e * N + n) * (K / 64) + d.k0 / 64 + j;
+    };
+    uint32_t sc_g = 0;  // stage the absmax cursor points at
+    if (total) srow = srow_of(0);
+    auto scale_next = [&]() -> float {
+      float v = 0.0f;
+      if (sc_g < total) {
+        if (srow) v = __ldg(srow + (int64_t)sc_cur.ks * BR * (K / 64));
+        ++sc_g;
+        if (++sc_cur.ks == NS) {
+          sc_cur.ks = 0;
+          ++sc_cur.tl;
+          if (sc_g < total) srow = srow_of(sc_cur.tl);
+        }
       }
-      const uint32_t ls = g % LS, bs = g % DS;
-      if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[ls], (g / LS) & 1u, abort, pb.err))) break;
+      return v;
+    };
+    float sA = scale_next(), sB = scale_next(), sC = scale_next(), sD = scale_next();
+    Cursor cur{0, 0};
+    bool jvalid = total ? dtile_info(blockIdx.x, off_s, ts_s, E).k0 + 64 * j < K : false;
+    uint32_t ls = 0, lph = 0, bs = 0, bph = 0;  // ring slots and parities of stage g
+    auto stage = [&](float a) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[ls], lph, abort, pb.err))) return false;
       // packed slab row n, bytes 32j .. 32j+31, stored 128B-swizzled
       const uint8_t* wst = smem + Smem::ld + ls * kLStageBytes + kAStageBytes + n * 128;
       const uint4 q0 = *reinterpret_cast<const uint4*>(wst + (((2 * j) ^ rr) << 4));
@@ -276,7 +284,7 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
       // overtake shared-memory loads still in flight
       __syncwarp();
       if (lane == 0) mbar_arrive(&ld_empty[ls]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&b_empty[bs], ((g / DS) & 1u) ^ 1u, abort, pb.err))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&b_empty[bs], bph ^ 1u, abort, pb.err))) return false;
       if (jvalid) {
         // K-row n of atom (n/8, j): 128 bytes, chunk c at (c ^ rr)
         uint8_t* dst = smem + Smem::b + bs * kBStageBytes + ((n >> 3) * 4 + j) * 1024 + rr * 128;
@@ -289,6 +297,30 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(&b_full[bs]);
+      // next stage
+      if (++ls == LS) { ls = 0; lph ^= 1u; }
+      if (++bs == DS) { bs = 0; bph ^= 1u; }
+      if (++cur.ks == NS) {
+        cur.ks = 0;
+        ++cur.tl;
+        if (cur.tl < my_tiles)
+          jvalid = dtile_info(blockIdx.x + cur.tl * gridDim.x, off_s, ts_s, E).k0 + 64 * j < K;
+      }
+      return true;
+    };
+    for (uint32_t g = 0; g < total;) {
+      if (!stage(sA)) break;
+      sA = scale_next();
+      if (++g >= total) break;
+      if (!stage(sB)) break;
+      sB = scale_next();
+      if (++g >= total) break;
+      if (!stage(sC)) break;
+      sC = scale_next();
+      if (++g >= total) break;
+      if (!stage(sD)) break;
+      sD = scale_next();
+      ++g;
     }
   } else if (warp >= 12) {
     // ---------------- epilogue ----------------
