@@ -16,7 +16,7 @@ import torch
 
 __all__ = [
     "lib", "GbwError", "gnf4_grouped_gemm", "gmxfp4_grouped_gemm",
-    "gnf4_grouped_dgrad", "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
+    "gnf4_grouped_dgrad", "gmxfp4_grouped_dgrad", "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
     "gmxfp4_quantize", "device_status", "MODE_AUTO", "MODE_GEMM", "MODE_GEMV",
     "DEVERR_OFFSETS", "DEVERR_TOKEN", "DEVERR_TIMEOUT", "FLAG_OVERLAP_PREV",
     "EXPORTS",
@@ -46,6 +46,7 @@ EXPORTS = {
     "gnf4_grouped_gemm": (C.c_int, [_P, _I64, _I64, _P, _P, _I32, _I64, _P, _P, _I64, _P, _I32, _P]),
     "gmxfp4_grouped_gemm": (C.c_int, [_P, _I64, _I64, _P, _P, _I32, _I64, _P, _P, _I64, _P, _I32, _P]),
     "gnf4_grouped_dgrad": (C.c_int, [_P, _I64, _I64, _P, _P, _I32, _I64, _P, _P, _P]),
+    "gmxfp4_grouped_dgrad": (C.c_int, [_P, _I64, _I64, _P, _P, _I32, _I64, _P, _P, _P]),
     "gnf4_dequant": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "gmxfp4_dequant": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "gnf4_quantize": (C.c_int, [_P, _I64, _I64, _P, _P, _P]),
@@ -170,6 +171,29 @@ def gnf4_grouped_dgrad(dy, packed, absmax, expert_offsets, out=None):
         _check(lib.gnf4_grouped_dgrad(_ptr(dy), P, N, _ptr(packed), _ptr(absmax),
                                       E, K, _ptr(expert_offsets), _ptr(out),
                                       _stream(dev)), "gnf4_grouped_dgrad")
+    return out
+
+
+def gmxfp4_grouped_dgrad(dy, blocks, scales, expert_offsets, out=None):
+    """dx[P, K] = dy[P, N] @ W_e per expert for MXFP4 weights (blocks
+    [E, N, K/32, 16] uint8, scales [E, N, K/32] uint8 e8m0)."""
+    _need(dy, "dy", torch.bfloat16)
+    dev = dy.device
+    _need(blocks, "blocks", torch.uint8, dev)
+    _need(scales, "scales", torch.uint8, dev)
+    _need(expert_offsets, "expert_offsets", torch.int32, dev)
+    P, N = dy.shape
+    E = blocks.shape[0]
+    K = blocks.shape[2] * 32 if blocks.dim() == 4 else blocks.shape[-1] * 2
+    if blocks.shape[1] != N:
+        raise ValueError("gmxfp4_grouped_dgrad: blocks rows must equal dy's N")
+    if out is None:
+        out = torch.empty((P, K), dtype=torch.bfloat16, device=dev)
+    _need(out, "dx", torch.bfloat16, dev)
+    with torch.cuda.device(dev):
+        _check(lib.gmxfp4_grouped_dgrad(_ptr(dy), P, N, _ptr(blocks), _ptr(scales),
+                                        E, K, _ptr(expert_offsets), _ptr(out),
+                                        _stream(dev)), "gmxfp4_grouped_dgrad")
     return out
 
 

@@ -141,31 +141,47 @@ gbw_status gmxfp4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
                          expert_offsets, row_to_token, P, out, mode, stream);
 }
 
-gbw_status gnf4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
-                              const uint8_t* packed, const float* absmax,
-                              int32_t E, int64_t K,
-                              const int32_t* expert_offsets, uint16_t* dx,
-                              void* stream) {
+static gbw_status grouped_dgrad(Fmt f, const uint16_t* dy, int64_t P, int64_t N,
+                                const uint8_t* packed, const void* scale, int32_t E,
+                                int64_t K, const int32_t* expert_offsets, uint16_t* dx,
+                                void* stream) {
   if (P < 0 || N <= 0 || K <= 0 || E < 1)
     return fail(GBW_ERR_SHAPE, "need P >= 0, N > 0, K > 0, E >= 1");
   if (K % 64 || N % 64) return fail(GBW_ERR_SHAPE, "dgrad needs K % 64 == 0 and N % 64 == 0");
   if (E > kMaxExperts) return fail(GBW_ERR_SHAPE, "at most 1024 experts");
   if (K > (int64_t)1 << 30 || P > INT32_MAX || (int64_t)E * N > INT32_MAX)
     return fail(GBW_ERR_SHAPE, "sizes exceed the 32-bit row indices");
-  if (!packed || !absmax || !expert_offsets) return fail(GBW_ERR_NULL, "NULL weights or offsets");
+  if (!packed || !scale || !expert_offsets) return fail(GBW_ERR_NULL, "NULL weights or offsets");
   if (P > 0 && (!dy || !dx)) return fail(GBW_ERR_NULL, "NULL dy or dx");
   if (!aligned16(dy) || !aligned16(packed) || !aligned16(dx))
     return fail(GBW_ERR_ALIGN, "dy, packed and dx must be 16-byte aligned");
-  if (!aligned4(absmax) || !aligned4(expert_offsets))
-    return fail(GBW_ERR_ALIGN, "absmax / offsets must be 4-byte aligned");
+  if ((f == Fmt::NF4 ? !aligned4(scale) : (reinterpret_cast<uintptr_t>(scale) & 1u) != 0) ||
+      !aligned4(expert_offsets))
+    return fail(GBW_ERR_ALIGN, "absmax 4-byte, scales 2-byte, offsets 4-byte aligned");
   int* err = nullptr;
   int sms = 0;
   gbw_status st = device_state(&err, &sms);
   if (st != GBW_OK) return st;
   if (P == 0) return GBW_OK;
-  GroupedProblem pb{dy, P, K, packed, absmax, E, N, expert_offsets, nullptr, P, dx, err, 0};
-  cudaError_t e = launch_dgrad(pb, sms, static_cast<cudaStream_t>(stream));
+  GroupedProblem pb{dy, P, K, packed, scale, E, N, expert_offsets, nullptr, P, dx, err, 0};
+  cudaError_t e = launch_dgrad(f, pb, sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GBW_OK : launch_error(e);
+}
+
+gbw_status gnf4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
+                              const uint8_t* packed, const float* absmax,
+                              int32_t E, int64_t K,
+                              const int32_t* expert_offsets, uint16_t* dx,
+                              void* stream) {
+  return grouped_dgrad(Fmt::NF4, dy, P, N, packed, absmax, E, K, expert_offsets, dx, stream);
+}
+
+gbw_status gmxfp4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
+                                const uint8_t* blocks, const uint8_t* scales,
+                                int32_t E, int64_t K,
+                                const int32_t* expert_offsets, uint16_t* dx,
+                                void* stream) {
+  return grouped_dgrad(Fmt::MXFP4, dy, P, N, blocks, scales, E, K, expert_offsets, dx, stream);
 }
 
 gbw_status gnf4_dequant(const uint8_t* packed, const float* absmax,

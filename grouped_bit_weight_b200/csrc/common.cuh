@@ -50,7 +50,7 @@ cudaError_t launch_gemv(Fmt f, const GroupedProblem& p, int num_sms,
 bool gemv_fits(Fmt f, const GroupedProblem& p, int num_sms);
 cudaError_t launch_gemm(Fmt f, const GroupedProblem& p, int num_sms,
                         cudaStream_t s);
-cudaError_t launch_dgrad(const GroupedProblem& p, int num_sms, cudaStream_t s);
+cudaError_t launch_dgrad(Fmt f, const GroupedProblem& p, int num_sms, cudaStream_t s);
 
 // ----------------------------------------------------------------------
 // device error word

@@ -1,10 +1,11 @@
-// dgrad.cu -- grouped NF4 activation gradient dx = dy * W on tcgen05.
+// dgrad.cu -- grouped 4-bit activation gradient dx = dy * W on tcgen05
+// (NF4 and MXFP4).
 //
 // "grouped-nf4-gemm 0.43.0", "Which entry point?": dgrad_4bit_grouped;
 // "Receipts-driven engineering": the NF4 path is differentiable and
 // fine-tuning never leaves the packed format.  For out = x W^T per expert,
 //   dx[p, k] = sum_n dy[p, n] * W_e(p)[n, k].
-// The reduction now runs over the weight rows n, and the absmax blocks lie
+// The reduction now runs over the weight rows n, and the scale blocks lie
 // along the output dimension k, so the weights are read packed in the
 // transposed orientation.
 //
@@ -101,6 +102,7 @@ struct AccSched {
   }
 };
 
+template <Fmt F>
 __global__ void __launch_bounds__(kThreads, 1)
 dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
              const __grid_constant__ CUtensorMap tmw) {
@@ -234,27 +236,35 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
     // bookkeeping is incremental: a cursor (local tile, stage) per
     // look-ahead distance steps one stage at a time and looks a tile up only
     // when it enters a new one (no divisions by the stage count), and the
-    // absmax of stage g + 4 is loaded into the slot stage g has just used
+    // scales of stage g + 4 are loaded into the slot stage g has just used
     // (fixed slots: a queue rotated by register copies would wait on each
     // load one stage after issuing it).
     struct Cursor {
       int64_t tl;
       int ks;
     };
-    // absmax cursor: the scale row of (weight row n, block j) in its tile
+    // scale cursor: the scales of (weight row n, block j) in its tile -- NF4
+    // one fp32 absmax per 64-k block, MXFP4 two e8m0 bytes (two 32-blocks)
     Cursor sc_cur{0, 0};
-    const float* srow = nullptr;  // absmax of weight row (e*N + n) at block k0/64 + j, or null
-    auto srow_of = [&](int64_t tl) -> const float* {
+    constexpr int kSB = F == Fmt::NF4 ? 4 : 2;           // scale bytes per 64-k block
+    const int64_t srow_bytes = F == Fmt::NF4 ? (K / 64) * 4 : K / 32;
+    const uint8_t* srow = nullptr;  // scales of weight row (e*N + n) at block j, or null
+    auto srow_of = [&](int64_t tl) -> const uint8_t* {
       const DTile d = dtile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E);
       if (d.k0 + 64 * j >= K) return nullptr;
-      return reinterpret_cast<const float*>(pb.scale) + ((int64_t)d.e * N + n) * (K / 64) + d.k0 / 64 + j;
+      return reinterpret_cast<const uint8_t*>(pb.scale) + ((int64_t)d.e * N + n) * srow_bytes +
+             (int64_t)(d.k0 / 64 + j) * kSB;
     };
-    uint32_t sc_g = 0;  // stage the absmax cursor points at
+    uint32_t sc_g = 0;  // stage the scale cursor points at
     if (total) srow = srow_of(0);
-    auto scale_next = [&]() -> float {
-      float v = 0.0f;
+    auto scale_next = [&]() -> uint32_t {
+      uint32_t v = 0u;
       if (sc_g < total) {
-        if (srow) v = __ldg(srow + (int64_t)sc_cur.ks * BR * (K / 64));
+        if (srow) {
+          const uint8_t* a = srow + (int64_t)sc_cur.ks * BR * srow_bytes;
+          v = F == Fmt::NF4 ? __ldg(reinterpret_cast<const uint32_t*>(a))
+                            : (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(a));
+        }
         ++sc_g;
         if (++sc_cur.ks == NS) {
           sc_cur.ks = 0;
@@ -264,11 +274,11 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
       }
       return v;
     };
-    float sA = scale_next(), sB = scale_next(), sC = scale_next(), sD = scale_next();
+    uint32_t sA = scale_next(), sB = scale_next(), sC = scale_next(), sD = scale_next();
     Cursor cur{0, 0};
     bool jvalid = total ? dtile_info(blockIdx.x, off_s, ts_s, E).k0 + 64 * j < K : false;
     uint32_t ls = 0, lph = 0, bs = 0, bph = 0;  // ring slots and parities of stage g
-    auto stage = [&](float a) -> bool {
+    auto stage = [&](uint32_t sv) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(&ld_full[ls], lph, abort, pb.err))) return false;
       // packed slab row n, bytes 32j .. 32j+31, stored 128B-swizzled
       const uint8_t* wst = smem + Smem::ld + ls * kLStageBytes + kAStageBytes + n * 128;
@@ -276,9 +286,19 @@ dgrad_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tma,
       const uint4 q1 = *reinterpret_cast<const uint4*>(wst + (((2 * j + 1) ^ rr) << 4));
       uint32_t o[32];
       const uint32_t P[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      const Planes tb = nf4_planes(a);
+      if (F == Fmt::NF4) {
+        const Planes tb = nf4_planes(__uint_as_float(sv));
 #pragma unroll
-      for (int i = 0; i < 8; ++i) decode_word<true>(P[i], tb, &o[4 * i]);
+        for (int i = 0; i < 8; ++i) decode_word<true>(P[i], tb, &o[4 * i]);
+      } else {
+        // two 32-blocks: bytes 0-15 (k 0..31) and 16-31 (k 32..63)
+        const Planes t0 = mxfp4_planes(sv & 0xFFu);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) decode_word<false>(P[i], t0, &o[4 * i]);
+        const Planes t1 = mxfp4_planes((sv >> 8) & 0xFFu);
+#pragma unroll
+        for (int i = 4; i < 8; ++i) decode_word<false>(P[i], t1, &o[4 * i]);
+      }
       // release the slab only once the decode has consumed what was loaded
       // from it: the refill is an async-proxy (TMA) write and must not
       // overtake shared-memory loads still in flight
@@ -376,7 +396,7 @@ cudaError_t make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
                         uint64_t d0, uint64_t d1, uint64_t pitch, uint32_t b0,
                         uint32_t b1, CUtensorMapSwizzle sw);
 
-cudaError_t launch_dgrad(const GroupedProblem& pb, int num_sms, cudaStream_t s) {
+cudaError_t launch_dgrad(Fmt f, const GroupedProblem& pb, int num_sms, cudaStream_t s) {
   if (pb.P == 0 || pb.K == 0) return cudaSuccess;
   CUtensorMap tma, tmw;
   // dy [P, N] bf16: box 64 (reduction) x 256 rows, 128B swizzle
@@ -392,10 +412,10 @@ cudaError_t launch_dgrad(const GroupedProblem& pb, int num_sms, cudaStream_t s) 
   static_assert(1024 + Smem::tables + 8 * (1024 + 1) <= 232448,
                 "shared memory for 1024 experts exceeds the 227 KB a CTA can have");
   const size_t smem = 1024 + Smem::tables + sizeof(int32_t) * 2 * (size_t)(pb.E + 1);
-  e = cudaFuncSetAttribute(dgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+  auto k = f == Fmt::NF4 ? dgrad_kernel<Fmt::NF4> : dgrad_kernel<Fmt::MXFP4>;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dgrad_kernel<<<num_sms, kThreads, smem, s>>>(pb, tma, tmw);
+  k<<<num_sms, kThreads, smem, s>>>(pb, tma, tmw);
   return cudaGetLastError();
 }
 

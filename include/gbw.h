@@ -127,6 +127,20 @@ GBW_API gbw_status gnf4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
                               const int32_t* expert_offsets, uint16_t* dx,
                               void* stream);
 
+/* Grouped MXFP4 activation gradient ("grouped-nf4-gemm 0.43.0", "Which
+ * entry point?": the MXFP4 entry point; "Receipts-driven engineering":
+ * training on the released MXFP4 bytes without requantisation).
+ *   dx[p, k] = bf16( sum_n dy[p, n] * W_e(p)[n, k] ),  fp32 accumulation
+ *   dy, dx, expert_offsets as in gnf4_grouped_dgrad; blocks / scales as in
+ *   gmxfp4_grouped_gemm (read packed, in the transposed orientation).
+ * Requires K % 64 == 0, N % 64 == 0, 16-byte aligned dy, blocks and dx,
+ * 2-byte aligned scales. */
+GBW_API gbw_status gmxfp4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
+                                const uint8_t* blocks, const uint8_t* scales,
+                                int32_t E, int64_t K,
+                                const int32_t* expert_offsets, uint16_t* dx,
+                                void* stream);
+
 /* Decode packed weights to bf16 ("grouped-nf4-gemm 0.43.0", "Try the
  * packers and byte checks on CPU", example 1: dequant_ref).  Bit-exact:
  * w[r, k] = bf16_rn(fp32(NF4[q] * absmax[r, k/64])).  rows counts all

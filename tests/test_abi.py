@@ -17,6 +17,7 @@ def _declared():
 def test_header_declares_the_entry_points():
     names = set(_declared())
     for n in ["gnf4_grouped_gemm", "gmxfp4_grouped_gemm", "gnf4_grouped_dgrad",
+              "gmxfp4_grouped_dgrad",
               "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
               "gmxfp4_quantize", "gbw_device_status", "gbw_status_string",
               "gbw_version"]:
@@ -72,6 +73,10 @@ def test_dgrad_and_codec_validation():
     assert L.gnf4_grouped_dgrad(p, 4, 60, p, p, 1, 128, p, p, None) == 2
     assert L.gnf4_grouped_dgrad(p, 4, 64, p, p, 1, 96, p, p, None) == 2
     assert L.gnf4_grouped_dgrad(None, 4, 64, p, p, 1, 128, p, p, None) == 1
+    assert L.gmxfp4_grouped_dgrad(p, 4, 60, p, p, 1, 128, p, p, None) == 2
+    assert L.gmxfp4_grouped_dgrad(p, 4, 64, p, p, 1, 96, p, p, None) == 2
+    assert L.gmxfp4_grouped_dgrad(None, 4, 64, p, p, 1, 128, p, p, None) == 1
+    assert L.gmxfp4_grouped_dgrad(p, 4, 64, p, C.c_void_p(17), 1, 128, p, p, None) == 3
     assert L.gnf4_dequant(p, p, 4, 96, p, None) == 2
     assert L.gmxfp4_dequant(p, p, 4, 48, p, None) == 2
     assert L.gnf4_quantize(None, 4, 64, p, p, None) == 1
