@@ -447,6 +447,33 @@ int orc_grouped_dgrad_sampled(const uint16_t* dy, int64_t P, int64_t N,
   return ORC_OK;
 }
 
+/* ------------------------------------------------------------------ */
+/* SwiGLU combine (the step between the two grouped matmuls of a fused  */
+/* expert pass)                                                          */
+/* ------------------------------------------------------------------ */
+
+/* The fused gate_up -> SwiGLU -> down expert pass ("Receipts-driven
+ * engineering", opening paragraph: the fused MoE path; the pages name the
+ * activation but print neither its formula nor the gate/up layout).
+ * Reading: the standard SwiGLU h = silu(gate) * up, silu(v) = v / (1 +
+ * exp(-v)), with gate = columns [0, I) and up = columns [I, 2I) of the bf16
+ * gate_up output, i.e. the gate_up weight stacks the gate rows above the up
+ * rows.  gu [P, 2I] bf16 -> h [P, I] bf16, evaluated in fp64 from the bf16
+ * inputs and rounded once to bf16 (the intermediate the down matmul reads). */
+int orc_swiglu(const uint16_t* gu, int64_t P, int64_t I, uint16_t* h) {
+  if (P < 0 || I <= 0) return ORC_ERR_SHAPE;
+#pragma omp parallel for schedule(static)
+  for (int64_t p = 0; p < P; ++p) {
+    const uint16_t* g = gu + p * 2 * I;
+    for (int64_t i = 0; i < I; ++i) {
+      const double gv = (double)bf16_to_f32(g[i]);
+      const double uv = (double)bf16_to_f32(g[I + i]);
+      h[p * I + i] = f64_to_bf16(gv / (1.0 + exp(-gv)) * uv);
+    }
+  }
+  return ORC_OK;
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -45,6 +45,7 @@ _sig("orc_grouped_forward_sampled", C.c_int, _P, _I64, _I64, _P, _I32, _I64,
 _sig("orc_grouped_dgrad", C.c_int, _P, _I64, _I64, _P, _I32, _I64, _P, _P, _P)
 _sig("orc_grouped_dgrad_sampled", C.c_int, _P, _I64, _I64, _P, _I32, _I64, _P,
      _P, _P, _I64, _P)
+_sig("orc_swiglu", C.c_int, _P, _I64, _I64, _P)
 _sig("orc_num_threads", C.c_int)
 _sig("orc_set_num_threads", None, C.c_int)
 
@@ -224,3 +225,26 @@ def grouped_dgrad_sampled(dy_bf16, wdec_bf16, offsets, sp, sk):
                                           sp.size, _ptr(out)),
            "grouped_dgrad_sampled")
     return out
+
+
+def swiglu(gu_bf16):
+    """SwiGLU combine of a fused gate_up output: gu [P, 2I] bf16 bits ->
+    h [P, I] bf16 bits, h = silu(gate) * up with gate = columns [0, I) and
+    up = columns [I, 2I) (the reading oracle.c states)."""
+    gu = _c(gu_bf16, np.uint16)
+    P, I2 = gu.shape
+    if I2 % 2:
+        raise OracleError("swiglu: gate_up width must be even")
+    h = np.empty((P, I2 // 2), np.uint16)
+    _check(_lib.orc_swiglu(_ptr(gu), P, I2 // 2, _ptr(h)), "swiglu")
+    return h
+
+
+def fused_expert(x_bf16, w_gate_up_bf16, w_down_bf16, offsets, row_to_token=None):
+    """One fused expert pass per routed row: the grouped gate_up matmul (bf16
+    out), the SwiGLU combine (bf16 h), then the grouped down matmul over the
+    same expert-sorted rows.  w_gate_up [E, 2I, H], w_down [E, H, I]."""
+    gu = grouped_forward(x_bf16, w_gate_up_bf16, offsets, row_to_token)
+    h = swiglu(gu)
+    return grouped_forward(h, w_down_bf16, offsets, None)
+

@@ -386,3 +386,78 @@ def test_hand_worked_grouped_matmul(fmt):
     out, o64 = orc.grouped_forward(x, wd, c["offsets"], c["row_to_token"], want_f64=True)
     assert np.array_equal(o64, c["out"])
     assert np.array_equal(bf16_bits_to_f64(out), c["out"])
+
+
+# ------------------------------------------------------- SwiGLU, fused pass
+
+def _bf16_bits(a64):
+    """fp64 -> bf16 bits with one rounding, by the oracle's f64_to_bf16,
+    which test_f64_to_bf16_is_nearest_with_ties_to_even pins by brute force
+    (torch's fp64 -> bf16 cast rounds twice, through fp32, so it cannot serve
+    as the reference here)."""
+    a = np.array(a64, np.float64)
+    return orc.f64_to_bf16(a.ravel()).reshape(a.shape)
+
+
+def test_swiglu_closed_forms():
+    """silu(0) = 0, silu(1) = 1 / (1 + e^-1), silu(-1) = -e^-1 / (1 + e^-1);
+    up = 0 gives 0; a large gate passes up through (silu(20) = 20 to bf16);
+    gate columns come first, up columns second."""
+    e1 = np.exp(-1.0)
+    gate = np.array([0.0, 1.0, -1.0, 3.0, 20.0, 1.0], np.float64)
+    up = np.array([5.0, 1.0, 1.0, 0.0, 0.5, 2.0], np.float64)
+    gu = _bf16_bits(np.concatenate([gate, up])[None, :])
+    h = bf16_bits_to_f64(orc.swiglu(gu))[0]
+    want = [0.0, 1.0 / (1.0 + e1), -e1 / (1.0 + e1), 0.0, 10.0, 2.0 / (1.0 + e1)]
+    got_bits = orc.swiglu(gu)[0]
+    assert np.array_equal(got_bits[[1, 2, 5]], _bf16_bits(np.array(want)[[1, 2, 5]]))
+    assert h[0] == 0.0 and h[3] == 0.0 and h[4] == 10.0
+    # swapping the halves changes the result: the layout is [gate | up]
+    swapped = _bf16_bits(np.concatenate([up, gate])[None, :])
+    assert not np.array_equal(orc.swiglu(swapped), orc.swiglu(gu))
+
+
+def test_swiglu_matches_torch_silu_in_fp64():
+    """Random bf16 gate/up values: h = bf16(silu(g) * u) with torch's silu in
+    fp64 (a library routine) and one rounding."""
+    rng = np.random.default_rng(11)
+    P, I = 37, 96
+    g = _bf16_bits(rng.standard_normal((P, I)) * 4)
+    u = _bf16_bits(rng.standard_normal((P, I)))
+    gu = np.concatenate([g, u], axis=1)
+    g64 = torch.from_numpy(bf16_bits_to_f64(g))
+    u64 = torch.from_numpy(bf16_bits_to_f64(u))
+    want = _bf16_bits((torch.nn.functional.silu(g64) * u64).numpy())
+    assert np.array_equal(orc.swiglu(gu), want)
+
+
+def test_fused_expert_brute_force():
+    """Fused pass on tiny shapes against an independent torch fp64 evaluation
+    with bf16 rounding at the two stated points (gate_up output, h); an
+    identity down projection returns h itself."""
+    rng = np.random.default_rng(12)
+    E, H, I, T = 3, 32, 16, 10
+    counts = np.array([4, 0, 7], np.int32)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    P = int(off[-1])
+    r2t = rng.integers(0, T, size=P).astype(np.int32)
+    x = _bf16_bits(rng.standard_normal((T, H)))
+    wgu = _bf16_bits(rng.standard_normal((E, 2 * I, H)) * 0.3)
+    wd = _bf16_bits(rng.standard_normal((E, H, I)) * 0.3)
+    got = orc.fused_expert(x, wgu, wd, off, r2t)
+    x64 = bf16_bits_to_f64(x)
+    want = np.zeros((P, H), np.uint16)
+    for e in range(E):
+        for p in range(off[e], off[e + 1]):
+            gu = _bf16_bits(bf16_bits_to_f64(wgu[e]) @ x64[r2t[p]])
+            g = torch.from_numpy(bf16_bits_to_f64(gu[:I]))
+            u = torch.from_numpy(bf16_bits_to_f64(gu[I:]))
+            h = _bf16_bits((torch.nn.functional.silu(g) * u).numpy())
+            want[p] = _bf16_bits(bf16_bits_to_f64(wd[e]) @ bf16_bits_to_f64(h))
+    assert np.array_equal(got, want)
+    # identity down projection (H = I): the pass returns the SwiGLU output
+    eye = _bf16_bits(np.array(np.broadcast_to(np.eye(I), (E, I, I))))
+    wgu_i = wgu[:, :, :I]
+    x_i = x[:, :I]
+    h_only = orc.swiglu(orc.grouped_forward(x_i, wgu_i, off, r2t))
+    assert np.array_equal(orc.fused_expert(x_i, wgu_i, eye, off, r2t), h_only)
