@@ -37,6 +37,17 @@ METRIC = "grouped 4-bit MoE GEMM TFLOP/s (prefill) and decode GB/s, % of B200 ro
 WORKLOAD = ("qwen3_30b_a3b_nf4_decode: E=128, top-8, 1 token; gate_up N=1536 K=2048 "
             "then down N=2048 K=768; weights N(0,0.02) NF4-packed, x N(0,1) bf16")
 N_SETS = 16  # disjoint 8-expert sets cycled by consecutive steps
+GRAPH_CHUNK = 1024  # layers per captured graph (a multiple of N_SETS)
+GU_CHAIN = 256      # gate_up launches per graph when timing that kernel alone
+
+
+def bench_config(world):
+    """The workload description both arms print (identical dicts)."""
+    return {"workload": WORKLOAD, "weights": "nf4 (absmax fp32 per 64)",
+            "activations": "bf16", "experts_cycled": f"{N_SETS} disjoint sets of 8",
+            "l2": "inputs larger than L2: 340 MB of packed weights cycled, 21 MB per step",
+            "path": "bandwidth GEMV (GBW_MODE_AUTO picks it for P <= 8)",
+            "parallelism": f"replicas x{world}"}
 
 
 def peaks():
@@ -186,7 +197,7 @@ def event_time_ms(torch, fn, iters, stream):
 
 def decode_routing(E, k, n_sets, seed):
     """Disjoint expert sets; set j routes one token to experts perm[k*j:k*(j+1)]."""
-    from grouped_bit_weight_b200 import synth
+    import synth
     perm = np.random.default_rng(seed).permutation(E)
     return [synth.decode_routing(E, k, 0, experts=np.sort(perm[k * j:k * (j + 1)]))
             for j in range(n_sets)]
@@ -195,7 +206,7 @@ def decode_routing(E, k, n_sets, seed):
 def run_ours(args, rank, world, dev):
     import torch
     import grouped_bit_weight_b200 as gbw
-    from grouped_bit_weight_b200 import synth
+    import synth
 
     hbm, bf16, bf16_sus, peak_kind = peaks()
     torch.cuda.set_device(dev)
@@ -234,24 +245,30 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize()
     assert gbw.device_status(dev) == 0
 
-    graphs = []
-    for j in range(N_SETS):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(j)
-        graphs.append(g)
-    cycle = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(cycle):
-        for j in range(N_SETS):
-            step(j)
+    # Exactly `n` layers, cycling the expert sets, as CUDA graphs of at most
+    # GRAPH_CHUNK layers (a multiple of N_SETS, so replays continue the
+    # cycle): the timed region is one graph launch for any --steps up to
+    # GRAPH_CHUNK, and the step count does not change the per-step cost.
+    def graphs_for(n):
+        out = []
+        for cnt, reps in ((GRAPH_CHUNK, n // GRAPH_CHUNK), (n % GRAPH_CHUNK, 1)):
+            if cnt and reps:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for j in range(cnt):
+                        step(j % N_SETS)
+                out.append((g, reps))
+        return out
 
-    def run_steps(n):
-        for _ in range(n // N_SETS):
-            cycle.replay()
-        for j in range(n % N_SETS):
-            graphs[j].replay()
+    warm_graphs = graphs_for(args.warmup)
+    timed_graphs = graphs_for(args.steps)
 
-    run_steps(args.warmup)
+    def run_graphs(gs):
+        for g, reps in gs:
+            for _ in range(reps):
+                g.replay()
+
+    run_graphs(warm_graphs)
     torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
@@ -261,7 +278,7 @@ def run_ours(args, rank, world, dev):
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        run_steps(args.steps)
+        run_graphs(timed_graphs)
         t1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
@@ -275,17 +292,19 @@ def run_ours(args, rank, world, dev):
     # one launch per expert set; average device time per launch
     gu_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gu_graph):
-        for j in range(N_SETS):
-            gbw.gnf4_grouped_gemm(x_gu, wgu[0], wgu[1], offs[j], r2ts[j], out=out_gu,
-                                  overlap_prev=True)
-    gu_ms = event_time_ms(torch, gu_graph.replay, 40, stream) / N_SETS
+        for j in range(GU_CHAIN):
+            gbw.gnf4_grouped_gemm(x_gu, wgu[0], wgu[1], offs[j % N_SETS], r2ts[j % N_SETS],
+                                  out=out_gu, overlap_prev=True)
+    gu_graph.replay()
+    gu_ms = event_time_ms(torch, gu_graph.replay, 4, stream) / GU_CHAIN
     launches["n"] += 0  # the roofline loop runs outside the timed region
     achieved = bytes_gu / (gu_ms * 1e-3) / 1e9
     traffic = load_traffic("gemv_nf4_qwen3_decode_gate_up")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                 "unit": "GB/s", "frac": round(achieved / hbm, 4),
                 "traffic": traffic, "kernel": "gemv_kernel<NF4> (gate_up)",
-                "timing": "graph of 16 back-to-back launches, CUDA events, per-launch mean",
+                "timing": f"graph of {GU_CHAIN} back-to-back launches cycling the 16 expert sets, "
+                          "replayed 4 times, CUDA events; per-launch mean",
                 "algorithmic_bytes_per_launch": bytes_gu,
                 "launch_ms": round(gu_ms, 5), "peak_source": peak_kind}
 
@@ -298,12 +317,9 @@ def run_ours(args, rank, world, dev):
         "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "weights": "nf4 (absmax fp32 per 64)",
-                   "activations": "bf16", "experts_cycled": f"{N_SETS} disjoint sets of 8",
-                   "l2": "inputs larger than L2: 340 MB of packed weights cycled, 21 MB per step",
-                   "path": "bandwidth GEMV (GBW_MODE_AUTO picks it for P <= 8)",
-                   "graphs": "steps replayed as CUDA graphs",
-                   "parallelism": f"replicas x{world}"},
+        "config": bench_config(world),
+        "timing": ("exactly --steps layers captured as CUDA graphs of up to "
+                   f"{GRAPH_CHUNK} layers, CUDA events on the launching stream"),
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": launches["n"],
@@ -336,7 +352,7 @@ def measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step, world
     """Same decode layer through the public API with host buffers: every step
     copies its inputs (x, offsets, row map) from pinned host memory and
     reads both outputs back; one synchronisation per step."""
-    from grouped_bit_weight_b200 import synth
+    import synth
     GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
     h_xgu = torch.randn((1, GU.K)).to(torch.bfloat16).pin_memory()
     h_xdn = torch.randn((8, DN.K)).to(torch.bfloat16).pin_memory()
@@ -471,7 +487,7 @@ def run_case(args, dev):
     profiling (ncu -k / -s / -c pick launches out of this command)."""
     import torch
     import grouped_bit_weight_b200 as gbw
-    from grouped_bit_weight_b200 import synth
+    import synth
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     gen = torch.Generator(device=dev)
@@ -540,7 +556,7 @@ def oracle_decode_step_fn():
     weights, then the fp64 grouped matmuls (inputs drawn on the CPU)."""
     sys.path.insert(0, os.path.join(ROOT, "oracle"))
     import oracle as orc
-    from grouped_bit_weight_b200 import synth
+    import synth
     GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
     pg = orc.nf4_pack(synth.normal((8, GU.N, GU.K), 31, GU.w_std))
     pd = orc.nf4_pack(synth.normal((8, DN.N, DN.K), 32, DN.w_std))
@@ -558,7 +574,7 @@ def oracle_decode_step_fn():
 
 
 def run_reference(args):
-    from grouped_bit_weight_b200 import synth
+    import synth
     GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
     step, cores = oracle_decode_step_fn()
     nbytes = gemv_bytes("nf4", 8, GU.N, GU.K, 1) + gemv_bytes("nf4", 8, DN.N, DN.K, 8)
@@ -575,7 +591,7 @@ def run_reference(args):
             "n_gpus": 1, "steps": n, "warmup": args.warmup,
             "ms_per_step": round(dt / n * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "runs_on": "host CPU cores"},
+            "config": bench_config(int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -583,8 +599,9 @@ def run_reference(args):
 
 
 def cpu_baseline():
-    """The oracle, as it stands, on ~10-30 s of the decode workload."""
-    from grouped_bit_weight_b200 import synth
+    """The oracle, as it stands, on ~10-30 s of the decode workload; plus the
+    tiny NF4 config on one thread (a 1-core figure)."""
+    import synth
     GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
     step, cores = oracle_decode_step_fn()
     nbytes = gemv_bytes("nf4", 8, GU.N, GU.K, 1) + gemv_bytes("nf4", 8, DN.N, DN.K, 8)
@@ -596,7 +613,38 @@ def cpu_baseline():
     dt = time.perf_counter() - t
     return {"value": round(nbytes * n / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
             "kind": "oracle",
-            "sample": f"{n} full decode layers (8 experts, gate_up + down) in {dt:.1f} s"}
+            "sample": f"{n} full decode layers (8 experts, gate_up + down) in {dt:.1f} s",
+            "tiny_single_thread": oracle_tiny_single_thread()}
+
+
+def oracle_tiny_single_thread():
+    """Config 1 (E=8, N=256, K=512, 64 tokens top-2 -> 128 routed rows) by
+    the oracle on one thread: NF4 decode of the 8 experts + fp64 grouped
+    forward, in GFLOP/s of 2*P*N*K."""
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import oracle as orc
+    import synth
+    off, r2t = synth.tiny_routing(0)
+    codes, absmax = orc.nf4_pack(synth.normal((8, 256, 512), 1))
+    x = synth.to_bf16_bits(synth.normal((64, 512), 2))
+    prev = orc.num_threads()
+    orc.set_num_threads(1)
+    try:
+        def one():
+            w = orc.nf4_decode(codes, absmax, 512, bf16=True)
+            orc.grouped_forward(x, w, off, r2t)
+        one()
+        n, t = 0, time.perf_counter()
+        while time.perf_counter() - t < 2.0:
+            one()
+            n += 1
+        dt = time.perf_counter() - t
+    finally:
+        orc.set_num_threads(prev)
+    flops = gemm_flops(int(off[-1]), 256, 512)
+    return {"value": round(flops * n / dt / 1e9, 4), "unit": "GFLOP/s", "cores": 1,
+            "ms_per_call": round(dt / n * 1e3, 3),
+            "sample": f"{n} calls of decode + grouped forward, tiny NF4 config"}
 
 
 # ---------------------------------------------------------------- main

@@ -81,17 +81,35 @@ def _stream(dev) -> C.c_void_p:
     return C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
 
 
-def _need(t, name, dtype, device=None):
+def _need(t, name, dtype):
+    """Type, dtype and layout of one argument (the device is checked by
+    _on_device once every size has been checked)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if device is not None and t.device != device:
-        raise ValueError(f"{name} is on {t.device}, expected {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _numel(t, name, n, where):
+    if t.numel() != n:
+        raise ValueError(f"{where}: {name} has {t.numel()} elements, needs {n}")
+
+
+def _on_device(where, **tensors):
+    """Every tensor is a CUDA tensor on one device; returns that device."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{where}: {name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{where}: {name} is on {t.device}, expected {dev}")
+    return dev
 
 
 _MODES = {"auto": MODE_AUTO, "gemm": MODE_GEMM, "gemv": MODE_GEMV}
@@ -100,26 +118,31 @@ _MODES = {"auto": MODE_AUTO, "gemm": MODE_GEMM, "gemv": MODE_GEMV}
 def _grouped(fn, where, x, w, scale, scale_dtype, expert_offsets, row_to_token,
              out, mode, K_div, overlap_prev=False):
     _need(x, "x", torch.bfloat16)
-    dev = x.device
-    _need(w, "packed weights", torch.uint8, dev)
-    _need(scale, "scales", scale_dtype, dev)
-    _need(expert_offsets, "expert_offsets", torch.int32, dev)
+    _need(w, "packed weights", torch.uint8)
+    _need(scale, "scales", scale_dtype)
+    _need(expert_offsets, "expert_offsets", torch.int32)
+    if x.dim() != 2 or w.dim() < 3:
+        raise ValueError(f"{where}: x must be [T, K] and the weights [E, N, ...]")
     T, K = x.shape
     E, N = w.shape[0], w.shape[1]
-    if w.numel() != E * N * (K // 2) or K % K_div:
-        raise ValueError(f"{where}: weights do not match x's K={K}")
-    if expert_offsets.numel() != E + 1:
-        raise ValueError(f"{where}: expert_offsets needs E+1={E + 1} entries")
+    if K % K_div:
+        raise ValueError(f"{where}: K={K} must be a multiple of {K_div}")
+    _numel(w, "packed weights", E * N * (K // 2), where)
+    _numel(scale, "scales", E * N * (K // (64 if K_div == 64 else 32)), where)
+    _numel(expert_offsets, "expert_offsets", E + 1, where)
     if row_to_token is not None:
-        _need(row_to_token, "row_to_token", torch.int32, dev)
+        _need(row_to_token, "row_to_token", torch.int32)
         P = row_to_token.numel()
     else:
         P = T
+    if out is not None:
+        _need(out, "out", torch.bfloat16)
+        if tuple(out.shape) != (P, N):
+            raise ValueError(f"{where}: out must be [{P}, {N}]")
+    dev = _on_device(where, x=x, w=w, scale=scale, expert_offsets=expert_offsets,
+                     row_to_token=row_to_token, out=out)
     if out is None:
         out = torch.empty((P, N), dtype=torch.bfloat16, device=dev)
-    _need(out, "out", torch.bfloat16, dev)
-    if tuple(out.shape) != (P, N):
-        raise ValueError(f"{where}: out must be [{P}, {N}]")
     m = _MODES[mode] if isinstance(mode, str) else int(mode)
     if overlap_prev:
         m |= FLAG_OVERLAP_PREV
@@ -151,107 +174,112 @@ def gmxfp4_grouped_gemm(x, blocks, scales, expert_offsets, row_to_token=None,
                     mode, 32, overlap_prev)
 
 
-def gnf4_grouped_dgrad(dy, packed, absmax, expert_offsets, out=None):
-    """dx[P, K] = dy[P, N] @ W_e per expert (the activation gradient of
-    gnf4_grouped_gemm, rows in the same expert-sorted order)."""
+def _dgrad(fn, where, dy, w, scale, scale_dtype, K, sdiv, expert_offsets, out):
     _need(dy, "dy", torch.bfloat16)
-    dev = dy.device
-    _need(packed, "packed", torch.uint8, dev)
-    _need(absmax, "absmax", torch.float32, dev)
-    _need(expert_offsets, "expert_offsets", torch.int32, dev)
+    _need(w, "packed weights", torch.uint8)
+    _need(scale, "scales", scale_dtype)
+    _need(expert_offsets, "expert_offsets", torch.int32)
+    if dy.dim() != 2 or w.dim() < 3:
+        raise ValueError(f"{where}: dy must be [P, N] and the weights [E, N, ...]")
     P, N = dy.shape
-    E = packed.shape[0]
-    K = packed.shape[-1] * 2
-    if packed.shape[1] != N:
-        raise ValueError("gnf4_grouped_dgrad: packed rows must equal dy's N")
+    E = w.shape[0]
+    if w.shape[1] != N:
+        raise ValueError(f"{where}: packed rows must equal dy's N={N}")
+    _numel(w, "packed weights", E * N * (K // 2), where)
+    _numel(scale, "scales", E * N * (K // sdiv), where)
+    _numel(expert_offsets, "expert_offsets", E + 1, where)
+    if out is not None:
+        _need(out, "dx", torch.bfloat16)
+        if tuple(out.shape) != (P, K):
+            raise ValueError(f"{where}: dx must be [{P}, {K}]")
+    dev = _on_device(where, dy=dy, w=w, scale=scale, expert_offsets=expert_offsets, out=out)
     if out is None:
         out = torch.empty((P, K), dtype=torch.bfloat16, device=dev)
-    _need(out, "dx", torch.bfloat16, dev)
     with torch.cuda.device(dev):
-        _check(lib.gnf4_grouped_dgrad(_ptr(dy), P, N, _ptr(packed), _ptr(absmax),
-                                      E, K, _ptr(expert_offsets), _ptr(out),
-                                      _stream(dev)), "gnf4_grouped_dgrad")
+        _check(fn(_ptr(dy), P, N, _ptr(w), _ptr(scale), E, K, _ptr(expert_offsets),
+                  _ptr(out), _stream(dev)), where)
     return out
+
+
+def gnf4_grouped_dgrad(dy, packed, absmax, expert_offsets, out=None):
+    """dx[P, K] = dy[P, N] @ W_e per expert (the activation gradient of
+    gnf4_grouped_gemm, rows in the same expert-sorted order); packed
+    [E, N, K/2] uint8, absmax [E, N, K/64] fp32."""
+    K = packed.shape[-1] * 2 if isinstance(packed, torch.Tensor) else 0
+    return _dgrad(lib.gnf4_grouped_dgrad, "gnf4_grouped_dgrad", dy, packed, absmax,
+                  torch.float32, K, 64, expert_offsets, out)
 
 
 def gmxfp4_grouped_dgrad(dy, blocks, scales, expert_offsets, out=None):
     """dx[P, K] = dy[P, N] @ W_e per expert for MXFP4 weights (blocks
-    [E, N, K/32, 16] uint8, scales [E, N, K/32] uint8 e8m0)."""
-    _need(dy, "dy", torch.bfloat16)
-    dev = dy.device
-    _need(blocks, "blocks", torch.uint8, dev)
-    _need(scales, "scales", torch.uint8, dev)
-    _need(expert_offsets, "expert_offsets", torch.int32, dev)
-    P, N = dy.shape
-    E = blocks.shape[0]
-    K = blocks.shape[2] * 32 if blocks.dim() == 4 else blocks.shape[-1] * 2
-    if blocks.shape[1] != N:
-        raise ValueError("gmxfp4_grouped_dgrad: blocks rows must equal dy's N")
+    [E, N, K/32, 16] or [E, N, K/2] uint8, scales [E, N, K/32] uint8 e8m0)."""
+    K = 0
+    if isinstance(blocks, torch.Tensor):
+        K = blocks.shape[2] * 32 if blocks.dim() == 4 else blocks.shape[-1] * 2
+    return _dgrad(lib.gmxfp4_grouped_dgrad, "gmxfp4_grouped_dgrad", dy, blocks, scales,
+                  torch.uint8, K, 32, expert_offsets, out)
+
+
+def _dequant(fn, where, w, scale, scale_dtype, K, sdiv, out_shape, out):
+    _need(w, "packed weights", torch.uint8)
+    _need(scale, "scales", scale_dtype)
+    if K <= 0 or K % sdiv:
+        raise ValueError(f"{where}: K={K} must be a positive multiple of {sdiv}")
+    rows = w.numel() // (K // 2)
+    _numel(w, "packed weights", rows * (K // 2), where)
+    _numel(scale, "scales", rows * (K // sdiv), where)
+    if out is not None:
+        _need(out, "out", torch.bfloat16)
+        _numel(out, "out", rows * K, where)
+    dev = _on_device(where, w=w, scale=scale, out=out)
     if out is None:
-        out = torch.empty((P, K), dtype=torch.bfloat16, device=dev)
-    _need(out, "dx", torch.bfloat16, dev)
+        out = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
     with torch.cuda.device(dev):
-        _check(lib.gmxfp4_grouped_dgrad(_ptr(dy), P, N, _ptr(blocks), _ptr(scales),
-                                        E, K, _ptr(expert_offsets), _ptr(out),
-                                        _stream(dev)), "gmxfp4_grouped_dgrad")
+        _check(fn(_ptr(w), _ptr(scale), rows, K, _ptr(out), _stream(dev)), where)
     return out
 
 
 def gnf4_dequant(packed, absmax, out=None):
-    """bf16 weights [..., K] decoded from NF4 (bit-exact)."""
-    _need(packed, "packed", torch.uint8)
-    dev = packed.device
-    _need(absmax, "absmax", torch.float32, dev)
+    """bf16 weights [..., K] decoded from NF4 packed [..., K/2] and absmax
+    [..., K/64] (bit-exact)."""
     K = packed.shape[-1] * 2
-    rows = packed.numel() // max(K // 2, 1)
-    if out is None:
-        out = torch.empty(packed.shape[:-1] + (K,), dtype=torch.bfloat16, device=dev)
-    _need(out, "out", torch.bfloat16, dev)
-    with torch.cuda.device(dev):
-        _check(lib.gnf4_dequant(_ptr(packed), _ptr(absmax), rows, K, _ptr(out),
-                                _stream(dev)), "gnf4_dequant")
-    return out
+    return _dequant(lib.gnf4_dequant, "gnf4_dequant", packed, absmax, torch.float32,
+                    K, 64, packed.shape[:-1] + (K,), out)
 
 
 def gmxfp4_dequant(blocks, scales, out=None):
-    """bf16 weights [..., K] decoded from MXFP4 blocks [..., K/32, 16]."""
-    _need(blocks, "blocks", torch.uint8)
-    dev = blocks.device
-    _need(scales, "scales", torch.uint8, dev)
-    K = blocks.shape[-2] * 32
-    rows = blocks.numel() // max(K // 2, 1)
-    if out is None:
-        out = torch.empty(blocks.shape[:-2] + (K,), dtype=torch.bfloat16, device=dev)
-    _need(out, "out", torch.bfloat16, dev)
-    with torch.cuda.device(dev):
-        _check(lib.gmxfp4_dequant(_ptr(blocks), _ptr(scales), rows, K, _ptr(out),
-                                  _stream(dev)), "gmxfp4_dequant")
-    return out
+    """bf16 weights [..., K] decoded from MXFP4 blocks [..., K/32, 16] and
+    scales [..., K/32]."""
+    K = blocks.shape[-2] * 32 if blocks.dim() >= 2 else 0
+    return _dequant(lib.gmxfp4_dequant, "gmxfp4_dequant", blocks, scales, torch.uint8,
+                    K, 32, blocks.shape[:-2] + (K,), out)
 
 
 def gnf4_quantize(w):
     """fp32 [..., K] -> (packed [..., K/2] uint8, absmax [..., K/64] fp32)."""
     _need(w, "w", torch.float32)
+    dev = _on_device("gnf4_quantize", w=w)
     K = w.shape[-1]
     rows = w.numel() // max(K, 1)
-    packed = torch.empty(w.shape[:-1] + (K // 2,), dtype=torch.uint8, device=w.device)
-    absmax = torch.empty(w.shape[:-1] + (K // 64,), dtype=torch.float32, device=w.device)
-    with torch.cuda.device(w.device):
+    packed = torch.empty(w.shape[:-1] + (K // 2,), dtype=torch.uint8, device=dev)
+    absmax = torch.empty(w.shape[:-1] + (K // 64,), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
         _check(lib.gnf4_quantize(_ptr(w), rows, K, _ptr(packed), _ptr(absmax),
-                                 _stream(w.device)), "gnf4_quantize")
+                                 _stream(dev)), "gnf4_quantize")
     return packed, absmax
 
 
 def gmxfp4_quantize(w):
     """fp32 [..., K] -> (blocks [..., K/32, 16] uint8, scales [..., K/32] uint8)."""
     _need(w, "w", torch.float32)
+    dev = _on_device("gmxfp4_quantize", w=w)
     K = w.shape[-1]
     rows = w.numel() // max(K, 1)
-    blocks = torch.empty(w.shape[:-1] + (K // 32, 16), dtype=torch.uint8, device=w.device)
-    scales = torch.empty(w.shape[:-1] + (K // 32,), dtype=torch.uint8, device=w.device)
-    with torch.cuda.device(w.device):
+    blocks = torch.empty(w.shape[:-1] + (K // 32, 16), dtype=torch.uint8, device=dev)
+    scales = torch.empty(w.shape[:-1] + (K // 32,), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
         _check(lib.gmxfp4_quantize(_ptr(w), rows, K, _ptr(blocks), _ptr(scales),
-                                   _stream(w.device)), "gmxfp4_quantize")
+                                   _stream(dev)), "gmxfp4_quantize")
     return blocks, scales
 
 

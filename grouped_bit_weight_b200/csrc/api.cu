@@ -4,20 +4,33 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace gbw {
 namespace {
 
-// GBW_DEVERR_* bits raised by the kernels of this library on this device.
+// GBW_DEVERR_* bits raised by the kernels of this library on this device,
+// and the copy of it that gbw_device_status takes atomically.
 __device__ int g_err_word;
+__device__ int g_err_copy;
 
 constexpr int kMaxDevices = 64;
 // Experts per call: the kernels keep expert_offsets in shared memory.
 constexpr int32_t kMaxExperts = 1024;
-int* g_err_ptr[kMaxDevices];
-int g_sms[kMaxDevices];
-int g_arch_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+
+// Per-device state, set up once per device (std::call_once, so host threads
+// that make their first calls at the same time see it complete).
+struct DeviceState {
+  int* err = nullptr;   // device address of g_err_word
+  int* copy = nullptr;  // device address of g_err_copy
+  int sms = 0;
+  int arch_ok = 0;      // 1 sm_100, -1 other
+  cudaError_t init = cudaSuccess;
+};
+DeviceState g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
 
 thread_local char g_msg[256] = "";
 
@@ -26,36 +39,49 @@ gbw_status launch_error(cudaError_t e) {
   return GBW_ERR_LAUNCH;
 }
 
-// Per-device state: architecture check, SM count and the device address of
-// the error word (resolved with the device current).
-gbw_status device_state(int** err, int* sms) {
+// Architecture check, SM count and the device addresses of the error word
+// and its copy (resolved with the device current).
+gbw_status device_state(int** err, int* sms, int** copy = nullptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return launch_error(e);
   if (dev < 0 || dev >= kMaxDevices) return GBW_ERR_ARCH;
-  if (g_arch_ok[dev] == 0) {
+  DeviceState& d = g_dev[dev];
+  std::call_once(g_dev_once[dev], [&]() {
     int major = 0, minor = 0, n = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (major != 10 || minor != 0) {
-      g_arch_ok[dev] = -1;
-    } else {
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_err_word);
-      if (e != cudaSuccess) return launch_error(e);
-      g_err_ptr[dev] = static_cast<int*>(p);
-      g_sms[dev] = n;
-      g_arch_ok[dev] = 1;
+      d.arch_ok = -1;
+      return;
     }
-  }
-  if (g_arch_ok[dev] < 0) {
+    void* p = nullptr;
+    void* c = nullptr;
+    d.init = cudaGetSymbolAddress(&p, g_err_word);
+    if (d.init == cudaSuccess) d.init = cudaGetSymbolAddress(&c, g_err_copy);
+    if (d.init != cudaSuccess) return;
+    d.err = static_cast<int*>(p);
+    d.copy = static_cast<int*>(c);
+    d.sms = n;
+    d.arch_ok = 1;
+  });
+  if (d.init != cudaSuccess) return launch_error(d.init);
+  if (d.arch_ok < 0) {
     snprintf(g_msg, sizeof(g_msg), "device %d is not sm_100 (B200)", dev);
     return GBW_ERR_ARCH;
   }
-  *err = g_err_ptr[dev];
-  *sms = g_sms[dev];
+  *err = d.err;
+  *sms = d.sms;
+  if (copy) *copy = d.copy;
   return GBW_OK;
+}
+
+// Takes the error word in one atomic step (and clears it when asked), so a
+// bit a kernel on another stream raises at the same time is either in the
+// copy or still in the word, never lost.
+__global__ void take_error_word(int* err, int* copy, int clear) {
+  *copy = clear ? atomicExch(err, 0) : atomicOr(err, 0);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -92,6 +118,8 @@ gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
   if (!aligned16(x) || !aligned16(w) || !aligned16(out))
     return fail(GBW_ERR_ALIGN, "x, packed weights and out must be 16-byte aligned");
   if (f == Fmt::NF4 && !aligned4(scale)) return fail(GBW_ERR_ALIGN, "absmax must be 4-byte aligned");
+  if (f == Fmt::MXFP4 && (reinterpret_cast<uintptr_t>(scale) & 1u))
+    return fail(GBW_ERR_ALIGN, "MXFP4 scales must be 2-byte aligned");
   if (!aligned4(offsets) || (row_to_token && !aligned4(row_to_token)))
     return fail(GBW_ERR_ALIGN, "offsets / row_to_token must be 4-byte aligned");
   if (mode == GBW_MODE_GEMM && K % 64)
@@ -246,18 +274,16 @@ gbw_status gmxfp4_quantize(const float* w, int64_t rows, int64_t K,
 
 gbw_status gbw_device_status(void* stream, int32_t* host_err, int32_t clear) {
   int* err = nullptr;
+  int* copy = nullptr;
   int sms = 0;
-  gbw_status st = device_state(&err, &sms);
+  gbw_status st = device_state(&err, &sms, &copy);
   if (st != GBW_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  take_error_word<<<1, 1, 0, s>>>(err, copy, clear ? 1 : 0);
+  cudaError_t e = cudaGetLastError();
   int v = 0;
-  cudaError_t e = cudaMemcpyAsync(&v, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&v, copy, sizeof(int), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e == cudaSuccess && clear && v) {
-    const int zero = 0;
-    e = cudaMemcpyAsync(err, &zero, sizeof(int), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  }
   if (e != cudaSuccess) return launch_error(e);
   if (host_err) *host_err = v;
   return v ? GBW_ERR_DEVICE : GBW_OK;

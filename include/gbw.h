@@ -104,7 +104,7 @@ GBW_API gbw_status gnf4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
  *   W_e[n, k] = e2m1(code) * 2^(scales[e, n, k/32] - 127)
  *   blocks [E, N, K/32, 16] uint8 (= [E, N, K/2]): byte j holds elements 2j
  *          (LOW nibble) and 2j+1 (high nibble); bit 3 of a code is its sign
- *   scales [E, N, K/32] uint8, e8m0 (0xFF is NaN)
+ *   scales [E, N, K/32] uint8, e8m0 (0xFF is NaN), 2-byte aligned
  * Everything else as gnf4_grouped_gemm; requires K % 32 == 0, N % 8 == 0. */
 GBW_API gbw_status gmxfp4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
                                const uint8_t* blocks, const uint8_t* scales,
@@ -170,9 +170,13 @@ GBW_API gbw_status gnf4_quantize(const float* w, int64_t rows, int64_t K,
 GBW_API gbw_status gmxfp4_quantize(const float* w, int64_t rows, int64_t K,
                            uint8_t* blocks, uint8_t* scales, void* stream);
 
-/* Reads the current device's error word (GBW_DEVERR_* bits) after
- * synchronising `stream`, stores it in *host_err, and clears it when
- * `clear` is non-zero.  Returns GBW_ERR_DEVICE when a bit is set. */
+/* Reads the current device's error word (GBW_DEVERR_* bits) on `stream`,
+ * stores it in *host_err, and clears it when `clear` is non-zero.  The word
+ * is taken in one atomic step on the device, so a bit that a kernel on
+ * another stream raises meanwhile is either returned or kept, never lost.
+ * Synchronises `stream`.  Returns GBW_ERR_DEVICE when a bit is set.  Calls
+ * for the same device from several host threads at once share one copy
+ * slot: serialise them. */
 GBW_API gbw_status gbw_device_status(void* stream, int32_t* host_err, int32_t clear);
 
 /* Static text for a status code; the last CUDA error text for

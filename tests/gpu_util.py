@@ -8,7 +8,7 @@ import numpy as np
 import torch
 
 import oracle as orc
-from grouped_bit_weight_b200 import synth
+import synth
 
 DEV = torch.device("cuda", 0)
 

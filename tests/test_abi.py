@@ -61,6 +61,10 @@ def test_host_validation_needs_no_gpu(fn):
     assert _call(fn, x=24) == ALIGN           # not 16-byte aligned
     assert _call(fn, out=8) == ALIGN
     if fn == "gnf4_grouped_gemm":
+        assert _call(fn, s=18) == ALIGN       # absmax needs 4-byte alignment
+    else:
+        assert _call(fn, s=17) == ALIGN       # e8m0 scales need 2-byte alignment
+    if fn == "gnf4_grouped_gemm":
         assert _call(fn, K=96) == SHAPE
     else:
         assert _call(fn, K=96, mode=1) == SHAPE  # tensor cores need K % 64

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle as orc
-from grouped_bit_weight_b200 import synth
+import synth
 
 pytestmark = pytest.mark.gpu
 

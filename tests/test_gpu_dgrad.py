@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 
 import oracle as orc
-from grouped_bit_weight_b200 import synth
+import synth
 from parity import assert_rows_close, assert_rows_exact_operands
 
 pytestmark = pytest.mark.gpu

@@ -11,7 +11,7 @@ pytestmark = pytest.mark.gpu
 
 gbw = pytest.importorskip("grouped_bit_weight_b200")
 from gpu_util import bits, to_dev  # noqa: E402
-from grouped_bit_weight_b200 import synth  # noqa: E402
+import synth  # noqa: E402
 
 
 @pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import oracle as orc
-from grouped_bit_weight_b200 import synth
+import synth
 from parity import assert_rows_close, assert_rows_exact_operands, check_rows
 
 pytestmark = pytest.mark.gpu

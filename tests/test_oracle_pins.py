@@ -9,7 +9,7 @@ import torch
 from scipy.stats import norm
 
 import oracle as orc
-from grouped_bit_weight_b200 import synth
+import synth
 from parity import bf16_bits_to_f64, check_rows
 
 # OCP MX v1.0, FP4 E2M1: the eight magnitudes, codes 0..7.
