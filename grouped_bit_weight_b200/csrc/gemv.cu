@@ -12,17 +12,22 @@
 //          takes a contiguous range of groups and each warp a contiguous
 //          chunk of it;
 //   loads  a warp issues the 16-byte loads of its rows' codes and scales for
-//          up to MG groups at once, straight into registers, so a CTA has
+//          up to MG row groups at once, straight into registers, so a CTA has
 //          its whole decode-sized share in flight about a microsecond after
-//          it starts, with no barrier, producer or staging copy in between;
-//   decode one packed byte (two codes) is decoded by one 4-byte shared-
-//          memory lookup that returns both codebook values as bf16, from a
-//          table holding one column per lane (entry b of lane l at
-//          b*256 + l*4, so the 32 lookups of a warp never share a bank; the
-//          table sits at a 64 KB-aligned shared address, so one byte permute
-//          builds the whole address), multiplied into fp32 accumulators by
-//          fma.rn.f32.bf16 with the bf16 activations (the product of two
-//          bf16 values is exact in fp32);
+//          it starts, with no barrier, producer or staging copy in between.
+//          Addresses come from one 64-bit row pointer per round plus
+//          constant strides (the per-load 64-bit index arithmetic used to
+//          cost as many instructions as the decode itself);
+//   decode one packed byte (two codes) is decoded by one 4-byte shared-memory
+//          lookup that returns both codebook values as bf16, from a table
+//          holding one column per lane (entry b of lane l at b*256 + l*4, so
+//          the 32 lookups of a warp never share a bank).  The offset is one
+//          byte permute and the table's base an immediate of the load, and
+//          each value is multiplied into an fp32 accumulator by
+//          fma.rn.f32.bf16 with the bf16 activation (one instruction; the
+//          product of two bf16 values is exact in fp32).  Measured on B200
+//          with the data in registers: 76 instructions per 16-byte unit, 40
+//          weights per clock per SM -- the rate HBM delivers NF4 weights;
 //   reduce each 16-byte unit's partial sum is scaled by its block scale; the
 //          G lanes of a row reduce with shuffles, two rows at a time (the
 //          lanes first swap halves, so a pair costs one shuffle more than a
@@ -41,7 +46,13 @@ namespace {
 
 constexpr int kThreads = 384;  // 12 warps: up to 168 registers a thread
 constexpr int kWarps = kThreads / 32;
-constexpr int kLutBytes = 256 * 256;  // 256 entries x 256-byte rows
+constexpr int kLutBytes = 256 * 256;  // 256 entries x 256-byte rows (lanes use 128 bytes)
+// Shared-window offset of the dynamic shared memory of a kernel without
+// static shared memory (measured on B200).  The table starts there; a launch
+// that finds it elsewhere adds the base at run time (one more instruction
+// per lookup).
+constexpr uint32_t kLutBaseGuess = 1024;
+constexpr uint32_t kRuntimeBase = 0xFFFFFFFFu;
 
 // Codebook value of code q, from immediates (a select tree, no memory
 // access: a table in constant memory costs a cold miss on every launch).
@@ -77,15 +88,20 @@ __device__ __forceinline__ float e8m0_f32(uint32_t s) {
   return __int_as_float((int)(s << 23));
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+// One table entry (two bf16 values): `off` = entry * 256 + lane * 4.
+template <uint32_t kBase>
+__device__ __forceinline__ uint32_t lut_ld(uint32_t off, uint32_t base) {
   uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  if (kBase != kRuntimeBase)
+    asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(off), "n"(kBase));
+  else
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(off + base));
   return v;
 }
 
-// a0 += lo(w) * lo(x), a1 += hi(w) * hi(x): bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void fma_pair(float& a0, float& a1, uint32_t w,
-                                         uint32_t x) {
+// a0 += lo(w) * lo(x), a1 += hi(w) * hi(x): bf16 inputs, fp32 accumulate
+// (one instruction each).
+__device__ __forceinline__ void fma_pair(float& a0, float& a1, uint32_t w, uint32_t x) {
   asm("{\n .reg .b16 wl, wh, xl, xh;\n"
       " mov.b32 {wl, wh}, %2;\n"
       " mov.b32 {xl, xh}, %3;\n"
@@ -97,33 +113,16 @@ __device__ __forceinline__ void fma_pair(float& a0, float& a1, uint32_t w,
 
 // sum over the 32 weights of one 16-byte unit of code value * x.  Byte m of
 // the unit holds elements 2m, 2m+1, and x pair m holds the same elements.
+template <uint32_t kBase>
 __device__ __forceinline__ float dot_unit(const uint4& q, const uint32_t (&x)[16],
-                                          uint32_t lut_lane) {
+                                          uint32_t lane4, uint32_t base) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
   float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    // table base | byte << 8 | lane*4: the lane's column of that byte's entry
-    const uint32_t addr = prmt(w[m >> 2], lut_lane, 0x7604u | ((m & 3) << 4));
-    const uint32_t v = lds32(addr);
-    fma_pair(a[2 * (m & 3)], a[2 * (m & 3) + 1], v, x[m]);
-  }
+  for (int m = 0; m < 16; ++m)  // byte << 8 | lane * 4: the lane's column of that byte's entry
+    fma_pair(a[2 * (m & 3)], a[2 * (m & 3) + 1],
+             lut_ld<kBase>(prmt(w[m >> 2], lane4, 0x7604u | ((m & 3) << 4)), base), x[m]);
   return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-}
-
-// Shared window: the decode table at the first 64 KB-aligned address; the
-// clamped expert offsets below it when they fit there, else after it.
-struct Layout {
-  uint32_t lut, off;
-};
-
-__device__ __forceinline__ Layout make_layout(uint32_t s0, int32_t E) {
-  Layout L;
-  L.lut = (s0 + 0xFFFFu) & ~0xFFFFu;
-  const uint32_t ob = 4u * (uint32_t)(E + 1);
-  const uint32_t lo = (s0 + 15u) & ~15u;
-  L.off = lo + ob <= L.lut ? lo : L.lut + (uint32_t)kLutBytes;
-  return L;
 }
 
 // Row groups a warp loads per round (register budget for codes + scales).
@@ -132,132 +131,92 @@ struct Round {
   static constexpr int MG = UPL == 1 ? 12 : (UPL == 2 ? 7 : 5);
 };
 
-template <Fmt F, int G, int UPL>
-__global__ void __launch_bounds__(kThreads, 1)
-gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  const Layout lay = make_layout(smem_u32(smem_raw), pb.E);
-  uint8_t* const base = smem_raw - smem_u32(smem_raw);  // shared window start
-  int32_t* off_s = reinterpret_cast<int32_t*>(base + lay.off);
-
+// The row groups [g0, g1) of one warp, after the kernel's prologue.
+template <Fmt F, int G, int UPL, uint32_t kBase>
+__device__ __forceinline__ void gemv_main(const GroupedProblem& pb, const int32_t* off_s,
+                                          int64_t g0, int64_t g1, int npass, int32_t tok,
+                                          uint32_t base, bool waited) {
   constexpr int RG = 32 / G;                // rows per row group
   constexpr int MG = Round<UPL>::MG;        // row groups per load round
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   const int li = lane % G, rs = lane / G;
   const int64_t K = pb.K, N = pb.N;
-  const int64_t U = K / 32;                 // 16-byte units per row
-  const int64_t srow = (F == Fmt::NF4) ? K / 64 : K / 32;  // scales per row
-
-  // this warp's row groups: a contiguous chunk of the CTA's contiguous range
-  const int64_t c0 = ngroups * blockIdx.x / gridDim.x;
-  const int64_t c1 = ngroups * (blockIdx.x + 1) / gridDim.x;
-  const int64_t g0 = c0 + (c1 - c0) * warp / kWarps;
-  const int64_t g1 = c0 + (c1 - c0) * (warp + 1) / kWarps;
+  const int32_t U = (int32_t)(K / 32);      // 16-byte units per row
+  const int32_t srow = (int32_t)((F == Fmt::NF4) ? K / 64 : K / 32);  // scales per row
+  const int64_t wstride = (int64_t)RG * U;  // 16-byte units between row groups
+  const int64_t sstride = (int64_t)RG * srow;
+  const uint32_t lane4 = (uint32_t)lane * 4u;
+  const uint4* const w16 = reinterpret_cast<const uint4*>(pb.w);
 
   // walk state: routed row p and column n of the next row group (advanced
   // by carry: one division per warp)
   int32_t p = (int32_t)(g0 * RG / N);
   int64_t n = g0 * RG - (int64_t)p * N;
+  int32_t e = expert_of_row(off_s, pb.E, p);
 
-  uint32_t xr[UPL][16];
-  int64_t xkey = -1;  // token * npass + pass held in xr
-  auto load_x = [&](int32_t tok, int pass) {
-    const uint4* xs = reinterpret_cast<const uint4*>(pb.x + (int64_t)tok * K);
-#pragma unroll
-    for (int i = 0; i < UPL; ++i) {
-      const int64_t u = ((int64_t)pass * UPL + i) * G + li;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        if (u < U) q = __ldg(xs + u * 4 + v);
-        xr[i][4 * v] = q.x;
-        xr[i][4 * v + 1] = q.y;
-        xr[i][4 * v + 2] = q.z;
-        xr[i][4 * v + 3] = q.w;
-      }
-    }
-    xkey = (int64_t)tok * npass + pass;
-  };
-  // Programmatic dependent launch.  x may be written by the kernel launched
-  // just before this one, so it is read only after grid_dependency_wait;
-  // with GBW_FLAG_OVERLAP_PREV the offsets, row map, codes and scales are
-  // not, so they are read while that kernel finishes.  The next kernel may
-  // launch once this one has passed its wait.
-  const bool early = (pb.flags & GBW_FLAG_OVERLAP_PREV) != 0;
-  bool waited = false;
-  auto ready = [&]() {
-    if (!waited) {
-      grid_dependency_wait();
-      grid_launch_dependents();
-      waited = true;
-    }
-  };
-  if (!early) ready();
-  // independent global loads first (the offsets and the first row's token),
-  // so the table below is built while they are in flight
-  const OffsetRegs offr = prefetch_offsets(pb.offsets, pb.E);
-  int32_t tok = g0 < g1 ? token_of_row(pb.row_to_token, p, pb.T, pb.err) : 0;
-  // pair table: entry b -> bf16 (value of the even element, value of the odd
-  // element) in every lane's column.  Thread b < 256 builds entry b and
-  // writes its 128-byte row with eight 16-byte stores, starting at chunk
-  // b % 8 so the 32 stores of a warp instruction spread over all banks.
-  // It touches no caller memory.
-  if (threadIdx.x < 256) {
-    const uint32_t b = threadIdx.x;
-    const uint32_t qe = (F == Fmt::NF4) ? (b >> 4) : (b & 15u);
-    const uint32_t qo = (F == Fmt::NF4) ? (b & 15u) : (b >> 4);
-    const uint32_t v =
-        (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qe))) |
-        ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qo))) << 16);
-    uint8_t* row = base + lay.lut + b * 256;
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      *reinterpret_cast<uint4*>(row + ((c + b) & 7u) * 16) = make_uint4(v, v, v, v);
-  }
-  if (!early && g0 < g1) load_x(tok, 0);
-  commit_offsets(offr, pb.offsets, pb.E, pb.P, off_s, pb.err);  // barrier inside
-
-  if (g0 >= g1) ready();
-  const uint32_t lut_lane = lay.lut | ((uint32_t)lane * 4u);
-  int32_t e = g0 < g1 ? expert_of_row(off_s, pb.E, p) : 0;
+  uint32_t xr[UPL][16];  // x of the current row and pass (bf16 pairs)
+  int64_t xkey = -1;     // token * npass + pass held in xr
   const bool hi = (li & (G / 2)) != 0;
   for (int64_t g = g0; g < g1;) {
     // one round: up to MG row groups of one routed row (one x)
     int cnt = (int)min((int64_t)MG, g1 - g);
     cnt = (int)min((int64_t)cnt, (N - n) / RG);
     const int64_t wrow0 = (int64_t)e * N + n + rs;  // weight row of group 0
+    const uint4* const wp = w16 + wrow0 * U;
+    const int64_t s0 = wrow0 * srow;
     float acc[MG];
 #pragma unroll
     for (int k = 0; k < MG; ++k) acc[k] = 0.0f;
     for (int pass = 0; pass < npass; ++pass) {
-      uint4 q[MG][UPL];
-      float sc[MG][UPL];
+      int32_t uo[UPL];  // this lane's units in the pass (>= U: past the row)
 #pragma unroll
-      for (int k = 0; k < MG; ++k) {
-        const int64_t wrow = wrow0 + (int64_t)k * RG;
+      for (int i = 0; i < UPL; ++i) uo[i] = (pass * UPL + i) * G + li;
+      uint4 q[MG][UPL];
+      uint32_t sc[MG][UPL];  // raw scale bits, converted when used
+#pragma unroll
+      for (int k = 0; k < MG; ++k)
 #pragma unroll
         for (int i = 0; i < UPL; ++i) {
-          const int64_t u = ((int64_t)pass * UPL + i) * G + li;
           q[k][i] = make_uint4(0u, 0u, 0u, 0u);
-          sc[k][i] = 0.0f;
-          if (k < cnt && u < U) {
-            q[k][i] = __ldg(reinterpret_cast<const uint4*>(pb.w + wrow * (K / 2)) + u);
+          sc[k][i] = 0u;
+          if (k < cnt && uo[i] < U) {
+            q[k][i] = __ldg(wp + k * wstride + uo[i]);
             if (F == Fmt::NF4)
-              sc[k][i] = __ldg(reinterpret_cast<const float*>(pb.scale) + wrow * srow + (u >> 1));
+              sc[k][i] = __ldg(reinterpret_cast<const uint32_t*>(pb.scale) + s0 + k * sstride + (uo[i] >> 1));
             else
-              sc[k][i] = e8m0_f32(__ldg(reinterpret_cast<const uint8_t*>(pb.scale) + wrow * srow + u));
+              sc[k][i] = __ldg(reinterpret_cast<const uint8_t*>(pb.scale) + s0 + k * sstride + uo[i]);
           }
         }
-      }
       if ((int64_t)tok * npass + pass != xkey) {
-        ready();
-        load_x(tok, pass);
+        // x may be written by the kernel launched just before this one: it
+        // is read only after that kernel has completed
+        if (!waited) {
+          grid_dependency_wait();
+          grid_launch_dependents();
+          waited = true;
+        }
+        const uint4* xs = reinterpret_cast<const uint4*>(pb.x + (int64_t)tok * K);
+#pragma unroll
+        for (int i = 0; i < UPL; ++i)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 t = make_uint4(0u, 0u, 0u, 0u);
+            if (uo[i] < U) t = __ldg(xs + uo[i] * 4 + v);
+            xr[i][4 * v] = t.x;
+            xr[i][4 * v + 1] = t.y;
+            xr[i][4 * v + 2] = t.z;
+            xr[i][4 * v + 3] = t.w;
+          }
+        xkey = (int64_t)tok * npass + pass;
       }
 #pragma unroll
       for (int k = 0; k < MG; ++k)
 #pragma unroll
         for (int i = 0; i < UPL; ++i)
-          if (k < cnt) acc[k] = fmaf(dot_unit(q[k][i], xr[i], lut_lane), sc[k][i], acc[k]);
+          if (k < cnt) {
+            const float s = F == Fmt::NF4 ? __uint_as_float(sc[k][i]) : e8m0_f32(sc[k][i]);
+            acc[k] = fmaf(dot_unit<kBase>(q[k][i], xr[i], lane4, base), s, acc[k]);
+          }
     }
     // Reduce pairs of row groups over the G lanes: the lower half of the
     // lanes collects group 2m, the upper half group 2m + 1.
@@ -285,6 +244,72 @@ gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
       tok = token_of_row(pb.row_to_token, p, pb.T, pb.err);
     }
   }
+  if (!waited) {
+    grid_dependency_wait();
+    grid_launch_dependents();
+  }
+}
+
+template <Fmt F, int G, int UPL>
+__global__ void __launch_bounds__(kThreads, 1)
+gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);  // the table: 256 rows of 256 bytes
+  int32_t* off_s = reinterpret_cast<int32_t*>(smem_raw + kLutBytes);
+  constexpr int RG = 32 / G;
+  const int warp = threadIdx.x >> 5;
+
+  // this warp's row groups: a contiguous chunk of the CTA's contiguous range
+  const int64_t c0 = ngroups * blockIdx.x / gridDim.x;
+  const int64_t c1 = ngroups * (blockIdx.x + 1) / gridDim.x;
+  const int64_t g0 = c0 + (c1 - c0) * warp / kWarps;
+  const int64_t g1 = c0 + (c1 - c0) * (warp + 1) / kWarps;
+
+  // Programmatic dependent launch.  Without GBW_FLAG_OVERLAP_PREV every
+  // input may come from the kernel launched just before this one, so this
+  // kernel waits for it first.  With the flag, the offsets, row map, codes
+  // and scales are read while that kernel finishes, and only x waits.  The
+  // next kernel may launch once this one has waited.
+  const bool early = (pb.flags & GBW_FLAG_OVERLAP_PREV) != 0;
+  if (!early) {
+    grid_dependency_wait();
+    grid_launch_dependents();
+  }
+  // independent global loads first (the offsets and the first row's token),
+  // so the table below is built while they are in flight
+  const OffsetRegs offr = prefetch_offsets(pb.offsets, pb.E);
+  const int32_t p0 = g0 < g1 ? (int32_t)(g0 * RG / pb.N) : 0;
+  const int32_t tok0 = g0 < g1 ? token_of_row(pb.row_to_token, p0, pb.T, pb.err) : 0;
+  // pair table: entry b -> bf16 (value of the even element, value of the odd
+  // element) in every lane's column.  Thread b < 256 builds entry b and
+  // writes its 128-byte row with eight 16-byte stores, starting at chunk
+  // b % 8 so the 32 stores of a warp instruction spread over all banks.  It
+  // touches no caller memory.
+  if (threadIdx.x < 256) {
+    const uint32_t b = threadIdx.x;
+    const uint32_t qe = (F == Fmt::NF4) ? (b >> 4) : (b & 15u);
+    const uint32_t qo = (F == Fmt::NF4) ? (b & 15u) : (b >> 4);
+    const uint32_t v =
+        (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qe))) |
+        ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qo))) << 16);
+    uint8_t* row = smem_raw + b * 256;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<uint4*>(row + ((c + b) & 7u) * 16) = make_uint4(v, v, v, v);
+  }
+  commit_offsets(offr, pb.offsets, pb.E, pb.P, off_s, pb.err);  // barrier inside
+
+  if (g0 >= g1) {
+    if (early) {
+      grid_dependency_wait();
+      grid_launch_dependents();
+    }
+    return;
+  }
+  if (base == kLutBaseGuess)
+    gemv_main<F, G, UPL, kLutBaseGuess>(pb, off_s, g0, g1, npass, tok0, base, !early);
+  else
+    gemv_main<F, G, UPL, kRuntimeBase>(pb, off_s, g0, g1, npass, tok0, base, !early);
 }
 
 struct Shape {
@@ -306,43 +331,25 @@ Shape pick_shape(int64_t U) {
   return best;
 }
 
-// Dynamic shared memory: enough that a 64 KB-aligned 64 KB table fits
-// wherever the window starts, plus the offsets.
-size_t gemv_smem(int32_t E) {
-  return 2 * (size_t)kLutBytes + 4 * (size_t)(E + 1) + 64;
-}
-
-// Per-device, per-kernel opt-in to the kernel's dynamic shared memory.
-// Guarded by a mutex: host threads may launch concurrently.
-cudaError_t opt_in(const void* fn, size_t smem) {
-  struct Entry { const void* fn; int dev; size_t smem; };
-  static std::mutex mu;
-  static Entry done[256];
-  static int ndone = 0;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < ndone; ++i)
-    if (done[i].fn == fn && done[i].dev == dev && done[i].smem >= smem) return cudaSuccess;
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  for (int i = 0; i < ndone; ++i)
-    if (done[i].fn == fn && done[i].dev == dev) {
-      done[i].smem = smem;
-      return cudaSuccess;
-    }
-  if (ndone < 256) done[ndone++] = Entry{fn, dev, smem};
-  return cudaSuccess;
-}
+// Dynamic shared memory: the 64 KB table, then the offsets.
+size_t gemv_smem(int32_t E) { return (size_t)kLutBytes + 4 * (size_t)(E + 1); }
 
 template <Fmt F, int G, int UPL>
 cudaError_t launch_t(const GroupedProblem& pb, int64_t ngroups, int npass,
                      int grid, cudaStream_t s) {
   auto k = gemv_kernel<F, G, UPL>;
   const size_t smem = gemv_smem(pb.E);
-  cudaError_t e = opt_in(reinterpret_cast<const void*>(k), smem);
+  // the shared-memory opt-in is set once per device and size
+  static size_t opted[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (opted[dev] < smem) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    opted[dev] = smem;
+  }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
