@@ -341,6 +341,10 @@ def run_ours(args, rank, world, dev):
     }
     if world == 1 and not args.no_secondary:
         result["secondary"] = secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind)
+        for e in result["secondary"]:  # the decode comparator against this layer's packed path
+            if e["workload"].startswith("comparator: dequantise-then-GEMM qwen3 decode layer"):
+                e["packed_ms"] = round(ms_per_step, 6)
+                e["packed_speedup"] = round(e["value"] / ms_per_step, 3)
         result["gpu_launches"] = launches["n"]
     return result
 
@@ -425,6 +429,27 @@ def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):
                              "peak": bf16, "unit": "TFLOP/s",
                              "frac": round(tf / bf16, 4), "peak_source": peak_kind}}
 
+    def hbm_entry(name, nbytes, ms, extra=None):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        e = {"workload": name, "value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 5),
+             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                          "unit": "GB/s", "frac": round(gbs / hbm, 4), "peak_source": peak_kind}}
+        if extra:
+            e.update(extra)
+        return e
+
+    def graph_ms(fn, n_inner, replays=20):
+        """Device time of fn() captured n_inner times in one CUDA graph, per
+        inner call (CUDA events around `replays` replays)."""
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n_inner):
+                fn()
+        g.replay()
+        return event_time_ms(torch, g.replay, replays, stream) / n_inner
+
     # Qwen3-30B-A3B prefill, NF4, tensor cores
     GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
     off, r2t = synth.prefill_routing()
@@ -432,29 +457,62 @@ def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):
     d_off = torch.from_numpy(off).to(dev)
     d_r2t = torch.from_numpy(r2t).to(dev)
     wgu = make_nf4(torch, gbw, GU.E, GU.N, GU.K, GU.w_std, gen, dev)
+    wdn = make_nf4(torch, gbw, DN.E, DN.N, DN.K, DN.w_std, gen, dev)
     x = torch.randn((4096, GU.K), generator=gen, device=dev).to(torch.bfloat16)
     o = torch.empty((P, GU.N), dtype=torch.bfloat16, device=dev)
-    out.append(tc_entry("qwen3 prefill gate_up NF4 (P=32768, N=1536, K=2048)",
-                        gemm_flops(P, GU.N, GU.K),
-                        lambda: gbw.gnf4_grouped_gemm(x, wgu[0], wgu[1], d_off, d_r2t, out=o)))
+    gu_prefill = tc_entry("qwen3 prefill gate_up NF4 (P=32768, N=1536, K=2048)",
+                          gemm_flops(P, GU.N, GU.K),
+                          lambda: gbw.gnf4_grouped_gemm(x, wgu[0], wgu[1], d_off, d_r2t, out=o))
+    out.append(gu_prefill)
     dy = (torch.randn((P, GU.N), generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
     dx = torch.empty((P, GU.K), dtype=torch.bfloat16, device=dev)
     out.append(tc_entry("qwen3 dgrad gate_up NF4 (P=32768, N=1536, K=2048)",
                         gemm_flops(P, GU.N, GU.K),
                         lambda: gbw.gnf4_grouped_dgrad(dy, wgu[0], wgu[1], d_off, out=dx)))
-    del wgu, x, o, dy, dx
-    wdn = make_nf4(torch, gbw, DN.E, DN.N, DN.K, DN.w_std, gen, dev)
+    del dy, dx
     xd = torch.randn((P, DN.K), generator=gen, device=dev).to(torch.bfloat16)
     od = torch.empty((P, DN.N), dtype=torch.bfloat16, device=dev)
-    out.append(tc_entry("qwen3 prefill down NF4 (P=32768, N=2048, K=768)",
-                        gemm_flops(P, DN.N, DN.K),
-                        lambda: gbw.gnf4_grouped_gemm(xd, wdn[0], wdn[1], d_off, None, out=od)))
+    dn_prefill = tc_entry("qwen3 prefill down NF4 (P=32768, N=2048, K=768)",
+                          gemm_flops(P, DN.N, DN.K),
+                          lambda: gbw.gnf4_grouped_gemm(xd, wdn[0], wdn[1], d_off, None, out=od))
+    out.append(dn_prefill)
     dyd = (torch.randn((P, DN.N), generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
     dxd = torch.empty((P, DN.K), dtype=torch.bfloat16, device=dev)
     out.append(tc_entry("qwen3 dgrad down NF4 (P=32768, N=2048, K=768)",
                         gemm_flops(P, DN.N, DN.K),
                         lambda: gbw.gnf4_grouped_dgrad(dyd, wdn[0], wdn[1], d_off, out=dxd)))
-    del wdn, xd, od, dyd, dxd
+    del dyd, dxd
+
+    # fused expert pass: gate_up with the SwiGLU epilogue, then down over h
+    hbuf = torch.empty((P, DN.K), dtype=torch.bfloat16, device=dev)
+    of = torch.empty((P, DN.N), dtype=torch.bfloat16, device=dev)
+    out.append(tc_entry("qwen3 prefill fused expert pass NF4 (gate_up + SwiGLU + down, P=32768)",
+                        gemm_flops(P, GU.N, GU.K) + gemm_flops(P, DN.N, DN.K),
+                        lambda: gbw.gnf4_grouped_expert_mlp(x, wgu[0], wgu[1], wdn[0], wdn[1], d_off,
+                                                            d_r2t, h=hbuf, out=of)))
+    sets = decode_routing(GU.E, 8, N_SETS, seed=5)
+    offs = [torch.from_numpy(a).to(dev) for a, _ in sets]
+    r2ts = [torch.from_numpy(b).to(dev) for _, b in sets]
+    x1 = torch.randn((1, GU.K), generator=gen, device=dev).to(torch.bfloat16)
+    h1 = torch.empty((8, DN.K), dtype=torch.bfloat16, device=dev)
+    o1 = torch.empty((8, DN.N), dtype=torch.bfloat16, device=dev)
+    it = {"j": 0}
+
+    def fused_decode():
+        j = it["j"] % N_SETS
+        it["j"] += 1
+        gbw.gnf4_grouped_expert_mlp(x1, wgu[0], wgu[1], wdn[0], wdn[1], offs[j], r2ts[j],
+                                    h=h1, out=o1)
+    ms = graph_ms(fused_decode, N_SETS)
+    out.append(hbm_entry("qwen3 decode fused expert pass NF4 (1 token, 8 experts; gate_up with "
+                         "SwiGLU then down, both on the bandwidth GEMV)",
+                         gemv_bytes("nf4", 8, GU.N, GU.K, 1) + gemv_bytes("nf4", 8, DN.N, DN.K, 8), ms))
+
+    # dequantise-then-GEMM comparator: decode the weights to bf16 in HBM
+    # (the library's bit-exact decoder), then cuBLAS bf16 matmuls per expert
+    out += dequant_comparator(torch, gbw, x, xd, wgu, wdn, off, r2t, d_r2t, sets, gu_prefill,
+                              dn_prefill, graph_ms, dev)
+    del wgu, wdn, x, o, xd, od, hbuf, of
     torch.cuda.empty_cache()
 
     # gpt-oss-20b MXFP4: 2048 tokens (tensor cores) and 1 token (GEMV)
@@ -468,6 +526,12 @@ def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):
         out.append(tc_entry(f"gpt-oss-20b {L.name.split('_')[-1]} MXFP4 batch 2048 (P=8192, N={L.N}, K={L.K})",
                             gemm_flops(P, L.N, L.K),
                             lambda: gbw.gmxfp4_grouped_gemm(x, w[0], w[1], d_off, d_r2t, out=o)))
+        dyg = (torch.randn((P, L.N), generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
+        dxg = torch.empty((P, L.K), dtype=torch.bfloat16, device=dev)
+        out.append(tc_entry(f"gpt-oss-20b {L.name.split('_')[-1]} MXFP4 dgrad batch 2048 (P=8192, N={L.N}, K={L.K})",
+                            gemm_flops(P, L.N, L.K),
+                            lambda: gbw.gmxfp4_grouped_dgrad(dyg, w[0], w[1], d_off, out=dxg)))
+        del dyg, dxg
         sets = decode_routing(L.E, 4, 8, seed=9)
         offs = [torch.from_numpy(a).to(dev) for a, _ in sets]
         r2ts = [torch.from_numpy(b).to(dev) for _, b in sets]
@@ -492,6 +556,70 @@ def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):
     torch.cuda.synchronize()
     assert gbw.device_status(dev) == 0
     return out
+
+
+def dequant_comparator(torch, gbw, x, xd, wgu, wdn, off, r2t, d_r2t, sets, gu_prefill,
+                       dn_prefill, graph_ms, dev):
+    """The pages' control experiment ("dequant tax"): the same projections
+    computed by first decoding the packed weights to bf16 in HBM
+    (gnf4_dequant, bit-exact), then bf16 matmuls by cuBLAS (torch.mm per
+    expert with routed rows, captured in one CUDA graph).  Reported next to
+    the packed path as time and the packed path's speedup."""
+    import synth
+    GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
+    res = []
+    cnt = np.diff(off)
+    live = [int(e) for e in np.nonzero(cnt)[0]]
+    P = int(off[-1])
+    # prefill: dequantise every expert of the layer (one launch), gather the
+    # routed rows, one matmul per expert with rows
+    r2t_long = d_r2t.long()
+    for L, w, xin, gathered, packed in ((GU, wgu, x, True, gu_prefill),
+                                        (DN, wdn, xd, False, dn_prefill)):
+        wbf = torch.empty((L.E, L.N, L.K), dtype=torch.bfloat16, device=dev)
+        xg = torch.empty((P, L.K), dtype=torch.bfloat16, device=dev)
+        ob = torch.empty((P, L.N), dtype=torch.bfloat16, device=dev)
+
+        def step():
+            gbw.gnf4_dequant(w[0], w[1], out=wbf)
+            src = xin
+            if gathered:
+                torch.index_select(xin, 0, r2t_long, out=xg)
+                src = xg
+            for e in live:
+                a, b = int(off[e]), int(off[e + 1])
+                torch.mm(src[a:b], wbf[e].t(), out=ob[a:b])
+        ms = graph_ms(step, 1, replays=10)
+        res.append({"workload": f"comparator: dequantise-then-GEMM qwen3 prefill {L.name.split('_')[-1]} "
+                                f"(gnf4_dequant of all {L.E} experts + {len(live)} cuBLAS bf16 matmuls)",
+                    "value": round(ms, 4), "unit": "ms", "higher_is_better": False,
+                    "packed_ms": packed["ms"], "packed_speedup": round(ms / packed["ms"], 3)})
+        del wbf, xg, ob
+    # decode layer: dequantise the 8 active experts of each projection, then
+    # batched matmuls (one token for gate_up, one row per expert for down)
+    wg8 = torch.empty((8, GU.N, GU.K), dtype=torch.bfloat16, device=dev)
+    wd8 = torch.empty((8, DN.N, DN.K), dtype=torch.bfloat16, device=dev)
+    x1 = torch.randn((1, 1, GU.K), device=dev).to(torch.bfloat16).expand(8, 1, GU.K)
+    xd8 = torch.randn((8, 1, DN.K), device=dev).to(torch.bfloat16)
+    og8 = torch.empty((8, 1, GU.N), dtype=torch.bfloat16, device=dev)
+    od8 = torch.empty((8, 1, DN.N), dtype=torch.bfloat16, device=dev)
+    experts = [[int(e) for e in np.nonzero(np.diff(o))[0]] for o, _ in sets]
+    it = {"j": 0}
+
+    def layer():
+        ex = experts[it["j"] % len(experts)]
+        it["j"] += 1
+        for i, e in enumerate(ex):
+            gbw.gnf4_dequant(wgu[0][e], wgu[1][e], out=wg8[i])
+            gbw.gnf4_dequant(wdn[0][e], wdn[1][e], out=wd8[i])
+        torch.bmm(x1, wg8.transpose(1, 2), out=og8)
+        torch.bmm(xd8, wd8.transpose(1, 2), out=od8)
+    ms = graph_ms(layer, len(experts))
+    res.append({"workload": "comparator: dequantise-then-GEMM qwen3 decode layer (16 gnf4_dequant "
+                            "launches for the 8 active experts of both projections + 2 cuBLAS "
+                            "batched bf16 matmuls)",
+                "value": round(ms, 5), "unit": "ms", "higher_is_better": False})
+    return res
 
 
 # ---------------------------------------------------------------- single cases

@@ -16,7 +16,8 @@ import torch
 
 __all__ = [
     "lib", "GbwError", "gnf4_grouped_gemm", "gmxfp4_grouped_gemm",
-    "gnf4_grouped_dgrad", "gmxfp4_grouped_dgrad", "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
+    "gnf4_grouped_dgrad", "gmxfp4_grouped_dgrad", "gnf4_grouped_expert_mlp",
+    "gmxfp4_grouped_expert_mlp", "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
     "gmxfp4_quantize", "device_status", "MODE_AUTO", "MODE_GEMM", "MODE_GEMV",
     "DEVERR_OFFSETS", "DEVERR_TOKEN", "DEVERR_TIMEOUT", "FLAG_OVERLAP_PREV",
     "EXPORTS",
@@ -47,6 +48,8 @@ EXPORTS = {
     "gmxfp4_grouped_gemm": (C.c_int, [_P, _I64, _I64, _P, _P, _I32, _I64, _P, _P, _I64, _P, _I32, _P]),
     "gnf4_grouped_dgrad": (C.c_int, [_P, _I64, _I64, _P, _P, _I32, _I64, _P, _P, _P]),
     "gmxfp4_grouped_dgrad": (C.c_int, [_P, _I64, _I64, _P, _P, _I32, _I64, _P, _P, _P]),
+    "gnf4_grouped_expert_mlp": (C.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _I32, _I64, _P, _P, _I64, _P, _P, _I32, _P]),
+    "gmxfp4_grouped_expert_mlp": (C.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _I32, _I64, _P, _P, _I64, _P, _P, _I32, _P]),
     "gnf4_dequant": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "gmxfp4_dequant": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "gnf4_quantize": (C.c_int, [_P, _I64, _I64, _P, _P, _P]),
@@ -218,6 +221,73 @@ def gmxfp4_grouped_dgrad(dy, blocks, scales, expert_offsets, out=None):
         K = blocks.shape[2] * 32 if blocks.dim() == 4 else blocks.shape[-1] * 2
     return _dgrad(lib.gmxfp4_grouped_dgrad, "gmxfp4_grouped_dgrad", dy, blocks, scales,
                   torch.uint8, K, 32, expert_offsets, out)
+
+
+def _expert_mlp(fn, where, x, gu, gu_scale, dn, dn_scale, scale_dtype, sdiv,
+                expert_offsets, row_to_token, h, out, mode):
+    _need(x, "x", torch.bfloat16)
+    for name, t in (("gate_up weights", gu), ("down weights", dn)):
+        _need(t, name, torch.uint8)
+    for name, t in (("gate_up scales", gu_scale), ("down scales", dn_scale)):
+        _need(t, name, scale_dtype)
+    _need(expert_offsets, "expert_offsets", torch.int32)
+    if x.dim() != 2 or gu.dim() < 3 or dn.dim() < 3:
+        raise ValueError(f"{where}: x must be [T, H] and the weights [E, rows, ...]")
+    T, H = x.shape
+    E, I2 = gu.shape[0], gu.shape[1]
+    I = I2 // 2
+    if I2 % 2 or dn.shape[0] != E or dn.shape[1] != H:
+        raise ValueError(f"{where}: gate_up must be [E, 2I, ...] and down [E, H={H}, ...]")
+    _numel(gu, "gate_up weights", E * I2 * (H // 2), where)
+    _numel(gu_scale, "gate_up scales", E * I2 * (H // sdiv), where)
+    _numel(dn, "down weights", E * H * (I // 2), where)
+    _numel(dn_scale, "down scales", E * H * (I // sdiv), where)
+    _numel(expert_offsets, "expert_offsets", E + 1, where)
+    if row_to_token is not None:
+        _need(row_to_token, "row_to_token", torch.int32)
+        P = row_to_token.numel()
+    else:
+        P = T
+    if h is not None:
+        _need(h, "h", torch.bfloat16)
+        if tuple(h.shape) != (P, I):
+            raise ValueError(f"{where}: h must be [{P}, {I}]")
+    if out is not None:
+        _need(out, "out", torch.bfloat16)
+        if tuple(out.shape) != (P, H):
+            raise ValueError(f"{where}: out must be [{P}, {H}]")
+    dev = _on_device(where, x=x, gu=gu, gu_scale=gu_scale, dn=dn, dn_scale=dn_scale,
+                     expert_offsets=expert_offsets, row_to_token=row_to_token, h=h, out=out)
+    if h is None:
+        h = torch.empty((P, I), dtype=torch.bfloat16, device=dev)
+    if out is None:
+        out = torch.empty((P, H), dtype=torch.bfloat16, device=dev)
+    m = _MODES[mode] if isinstance(mode, str) else int(mode)
+    with torch.cuda.device(dev):
+        _check(fn(_ptr(x), T, H, _ptr(gu), _ptr(gu_scale), _ptr(dn), _ptr(dn_scale), E, I,
+                  _ptr(expert_offsets), _ptr(row_to_token), P, _ptr(h), _ptr(out), m,
+                  _stream(dev)), where)
+    return out, h
+
+
+def gnf4_grouped_expert_mlp(x, gu_packed, gu_absmax, dn_packed, dn_absmax, expert_offsets,
+                            row_to_token=None, h=None, out=None, mode="auto"):
+    """Fused expert pass: gate_up [E, 2I, H/2] (gate rows then up rows),
+    h = silu(gate) * up [P, I] (workspace, returned), down [E, H, I/2] ->
+    out [P, H].  Returns (out, h).  mode "auto": both projections on the
+    bandwidth GEMV when P <= 8, else both on the tensor cores."""
+    return _expert_mlp(lib.gnf4_grouped_expert_mlp, "gnf4_grouped_expert_mlp", x, gu_packed,
+                       gu_absmax, dn_packed, dn_absmax, torch.float32, 64, expert_offsets,
+                       row_to_token, h, out, mode)
+
+
+def gmxfp4_grouped_expert_mlp(x, gu_blocks, gu_scales, dn_blocks, dn_scales, expert_offsets,
+                              row_to_token=None, h=None, out=None, mode="auto"):
+    """MXFP4 fused expert pass (blocks [E, rows, K/32, 16], e8m0 scales
+    [E, rows, K/32]).  Returns (out, h)."""
+    return _expert_mlp(lib.gmxfp4_grouped_expert_mlp, "gmxfp4_grouped_expert_mlp", x, gu_blocks,
+                       gu_scales, dn_blocks, dn_scales, torch.uint8, 32, expert_offsets,
+                       row_to_token, h, out, mode)
 
 
 def _dequant(fn, where, w, scale, scale_dtype, K, sdiv, out_shape, out):

@@ -212,6 +212,72 @@ gbw_status gmxfp4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N,
   return grouped_dgrad(Fmt::MXFP4, dy, P, N, blocks, scales, E, K, expert_offsets, dx, stream);
 }
 
+static gbw_status expert_mlp(Fmt f, const uint16_t* x, int64_t T, int64_t H,
+                             const uint8_t* gu, const void* gu_scale, const uint8_t* dn,
+                             const void* dn_scale, int32_t E, int64_t I,
+                             const int32_t* offsets, const int32_t* row_to_token, int64_t P,
+                             uint16_t* h, uint16_t* out, int32_t mode, void* stream) {
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || P < 0)
+    return fail(GBW_ERR_SHAPE, "need T >= 0, H > 0, I > 0, E >= 1, P >= 0");
+  if (H % 64 || I % 64)
+    return fail(GBW_ERR_SHAPE, "the fused expert pass needs H % 64 == 0 and I % 64 == 0");
+  if (H > (int64_t)1 << 30 || I > (int64_t)1 << 29 || P > INT32_MAX || T > INT32_MAX ||
+      (int64_t)E * 2 * I > INT32_MAX || (int64_t)E * H > INT32_MAX)
+    return fail(GBW_ERR_SHAPE, "sizes exceed the 32-bit row indices");
+  if (mode < GBW_MODE_AUTO || mode > GBW_MODE_GEMV)
+    return fail(GBW_ERR_SHAPE, "unknown mode (the fused pass takes no flags)");
+  if (E > kMaxExperts) return fail(GBW_ERR_SHAPE, "at most 1024 experts");
+  if (!offsets || !gu || !gu_scale || !dn || !dn_scale)
+    return fail(GBW_ERR_NULL, "NULL weights or offsets");
+  if (P > 0 && (!x || !h || !out)) return fail(GBW_ERR_NULL, "NULL x, h or out");
+  if (!row_to_token && T < P) return fail(GBW_ERR_SHAPE, "row_to_token == NULL needs T >= P");
+  if (row_to_token && P > 0 && T < 1) return fail(GBW_ERR_SHAPE, "T must be >= 1");
+  if (!aligned16(x) || !aligned16(gu) || !aligned16(dn) || !aligned16(h) || !aligned16(out))
+    return fail(GBW_ERR_ALIGN, "x, packed weights, h and out must be 16-byte aligned");
+  if (f == Fmt::NF4 && (!aligned4(gu_scale) || !aligned4(dn_scale)))
+    return fail(GBW_ERR_ALIGN, "absmax must be 4-byte aligned");
+  if (f == Fmt::MXFP4 && ((reinterpret_cast<uintptr_t>(gu_scale) | reinterpret_cast<uintptr_t>(dn_scale)) & 1u))
+    return fail(GBW_ERR_ALIGN, "MXFP4 scales must be 2-byte aligned");
+  if (!aligned4(offsets) || (row_to_token && !aligned4(row_to_token)))
+    return fail(GBW_ERR_ALIGN, "offsets / row_to_token must be 4-byte aligned");
+  int* err = nullptr;
+  int sms = 0;
+  gbw_status st = device_state(&err, &sms);
+  if (st != GBW_OK) return st;
+  if (P == 0) return GBW_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // gate_up with SwiGLU fused into the output (h = silu(gate) * up), then
+  // down over h (row p of h is routed row p); both on the bandwidth GEMV or
+  // both on the tensor cores
+  const bool gemv = mode == GBW_MODE_GEMV || (mode == GBW_MODE_AUTO && P <= 8);
+  GroupedProblem g{x, T, H, gu, gu_scale, E, 2 * I, offsets, row_to_token, P, h, err, 0};
+  cudaError_t e = gemv ? launch_gemv(f, g, sms, s, true) : launch_gemm(f, g, sms, s, I);
+  if (e != cudaSuccess) return launch_error(e);
+  GroupedProblem d{h, P, I, dn, dn_scale, E, H, offsets, nullptr, P, out, err, 0};
+  e = gemv ? launch_gemv(f, d, sms, s) : launch_gemm(f, d, sms, s);
+  return e == cudaSuccess ? GBW_OK : launch_error(e);
+}
+
+gbw_status gnf4_grouped_expert_mlp(const uint16_t* x, int64_t T, int64_t H,
+                                   const uint8_t* gu_packed, const float* gu_absmax,
+                                   const uint8_t* dn_packed, const float* dn_absmax,
+                                   int32_t E, int64_t I, const int32_t* expert_offsets,
+                                   const int32_t* row_to_token, int64_t P, uint16_t* h,
+                                   uint16_t* out, int32_t mode, void* stream) {
+  return expert_mlp(Fmt::NF4, x, T, H, gu_packed, gu_absmax, dn_packed, dn_absmax, E, I,
+                    expert_offsets, row_to_token, P, h, out, mode, stream);
+}
+
+gbw_status gmxfp4_grouped_expert_mlp(const uint16_t* x, int64_t T, int64_t H,
+                                     const uint8_t* gu_blocks, const uint8_t* gu_scales,
+                                     const uint8_t* dn_blocks, const uint8_t* dn_scales,
+                                     int32_t E, int64_t I, const int32_t* expert_offsets,
+                                     const int32_t* row_to_token, int64_t P, uint16_t* h,
+                                     uint16_t* out, int32_t mode, void* stream) {
+  return expert_mlp(Fmt::MXFP4, x, T, H, gu_blocks, gu_scales, dn_blocks, dn_scales, E, I,
+                    expert_offsets, row_to_token, P, h, out, mode, stream);
+}
+
 gbw_status gnf4_dequant(const uint8_t* packed, const float* absmax,
                         int64_t rows, int64_t K, uint16_t* w_out,
                         void* stream) {

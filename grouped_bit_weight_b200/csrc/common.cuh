@@ -44,12 +44,16 @@ cudaError_t launch_dequant(Fmt f, const uint8_t* w, const void* scale,
                            cudaStream_t s);
 cudaError_t launch_quantize(Fmt f, const float* w, int64_t rows, int64_t K,
                             uint8_t* codes, void* scale, cudaStream_t s);
+// glu: the SwiGLU gate_up variant (p.N = 2I rows per expert, gate rows then
+// up rows); out receives h = silu(gate) * up, [P, I].
 cudaError_t launch_gemv(Fmt f, const GroupedProblem& p, int num_sms,
-                        cudaStream_t s);
+                        cudaStream_t s, bool glu = false);
 // Whether the GEMV's shared-memory ring holds two blocks of rows of length K.
 bool gemv_fits(Fmt f, const GroupedProblem& p, int num_sms);
+// glu_i > 0: the SwiGLU gate_up variant (p.N = 2 * glu_i rows per expert,
+// gate rows then up rows); out receives h = silu(gate) * up, [P, glu_i].
 cudaError_t launch_gemm(Fmt f, const GroupedProblem& p, int num_sms,
-                        cudaStream_t s);
+                        cudaStream_t s, int64_t glu_i = 0);
 cudaError_t launch_dgrad(Fmt f, const GroupedProblem& p, int num_sms, cudaStream_t s);
 
 // ----------------------------------------------------------------------

@@ -39,6 +39,14 @@
 // Tensor memory holds two 128 x 256 fp32 accumulator halves: tiles of up to
 // 256 rows alternate between them, so the epilogue of one overlaps the
 // mainloop of the next; a wider tile takes both.
+// SwiGLU variant (the gate_up projection of the fused expert pass): a tile
+// holds 64 gate rows and the matching 64 up rows (two TMA boxes), and each
+// decode thread writes gate row j to A-tile row 32*(j/16) + j%16 and up row
+// j sixteen rows further.  Gate and up of one output column then land in
+// TMEM lanes l and l + 16 of one epilogue warp, which pairs them with one
+// shuffle and writes h = bf16(silu(bf16 gate) * bf16 up) -- no cross-warp
+// exchange, and the decoded rows of a quarter-warp stay consecutive (no
+// bank conflicts on the swizzled A-tile stores).
 // Scheduler: tiles (expert, 128-row weight tile, token tile) with
 // zero-row experts skipped, enumerated from expert_offsets by every CTA and
 // dealt round-robin (token tiles innermost, so CTAs running at the same time
@@ -121,7 +129,8 @@ struct TileInfo {
 };
 
 __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
-                                              const int32_t* ts, int32_t E, int32_t BT) {
+                                              const int32_t* ts, int32_t E, int32_t BT,
+                                              int32_t NS = BM) {
   int32_t lo = 0, hi = E - 1;  // last e with ts[e] <= t
   while (lo < hi) {
     int32_t mid = (lo + hi + 1) >> 1;
@@ -133,18 +142,22 @@ __device__ __forceinline__ TileInfo tile_info(int64_t t, const int32_t* off,
   const int32_t nt = u / tt, mt = u - nt * tt;
   TileInfo ti;
   ti.e = lo;
-  ti.n0 = nt * BM;
+  ti.n0 = nt * NS;
   ti.p0 = off[lo] + mt * BT;
   ti.nv = min(BT, cnt - mt * BT);
   return ti;
 }
 
-template <Fmt F, bool W>
+template <Fmt F, bool W, bool kGLU>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
             const __grid_constant__ CUtensorMap tmx32,
-            const __grid_constant__ CUtensorMap tmw, const int srow,
-            const int tile_scales) {
+            const __grid_constant__ CUtensorMap tmw,
+            const __grid_constant__ CUtensorMap tmw64, const int srow,
+            const int tile_scales, const int32_t glu_i) {
+  // kGLU: pb.N = 2 * glu_i weight rows per expert (gate rows, then up rows);
+  // a tile covers NS = 64 gate columns; out is h [P, glu_i]
+  constexpr int NS = kGLU ? 64 : BM;
   constexpr int BT = TileCfg<W>::BT;  // routed rows per tile
   constexpr int XS = TileCfg<W>::XS;  // activation ring stages
   constexpr int kXStageBytes = TileCfg<W>::kXStageBytes;
@@ -173,7 +186,8 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
   const int32_t E = pb.E;
   const int64_t K = pb.K, N = pb.N;
   const int NK = (int)(K / BK);
-  const int32_t ntn = (int32_t)((N + BM - 1) / BM);
+  const int32_t ntn = kGLU ? glu_i / NS : (int32_t)((N + BM - 1) / BM);
+  const int64_t ON = kGLU ? (int64_t)glu_i : N;  // columns of out
   const bool gathered = pb.row_to_token != nullptr;
 
   if (threadIdx.x == 0) {
@@ -196,7 +210,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     tma_prefetch_desc(&tmx);
     tma_prefetch_desc(&tmx32);
   }
-  if ((warp == 4 || warp == 8) && lane == 0) tma_prefetch_desc(&tmw);
+  if ((warp == 4 || warp == 8) && lane == 0) tma_prefetch_desc(kGLU ? &tmw64 : &tmw);
   load_offsets_clamped(pb.offsets, E, pb.P, off_s, pb.err);  // has __syncthreads
   tile_prefix(off_s, E, BT, ntn, ts_s);
   tc_fence_before();
@@ -215,7 +229,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       // a partial half uses (most experts end in a partial tile)
       if (warp == 2 && lane == 0) {
         for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-          const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
+          const TileInfo ti = tile_info(t, off_s, ts_s, E, BT, NS);
           for (int kb = 0; kb < NK; ++kb, ++g) {
             const uint32_t s = g % XS, ph = (g / XS) & 1u;
             if (!(ok = mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err))) break;
@@ -256,7 +270,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       const int chunk = lane & 7;
       const int r0 = 4 * gw + (lane >> 3);
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
+        const TileInfo ti = tile_info(t, off_s, ts_s, E, BT, NS);
         int32_t tk[kRows];
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
@@ -293,7 +307,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       const uint64_t adesc0 = make_sdesc_sw128(smem_u32(smem + Smem::a), 16, 1024);
       AccSched acc;
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
+        const TileInfo ti = tile_info(t, off_s, ts_s, E, BT, NS);
         const bool wide = ti.nv > BH;
         const uint32_t h0 = acc.h, h1 = acc.h ^ 1u;
         const uint32_t idesc0 = make_idesc_bf16(BM, wide ? (uint32_t)BH : (uint32_t)((ti.nv + 15) & ~15), 0, 0);
@@ -352,7 +366,10 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     const uint32_t grp = (uint32_t)(warp - 4) >> 2;
     const uint32_t q = (uint32_t)warp & 3u;
     const int m = (int)(q * 32 + lane);              // weight row in tile
-    const int mr = m & 7;                            // row inside its 8-row atom
+    // A-tile row of weight row m: SwiGLU puts gate j at 32*(j/16) + j%16 and
+    // up j sixteen rows further (lanes l and l + 16 of one epilogue warp)
+    const int ar = kGLU ? ((m & 63) >> 4) * 32 + ((m >> 6) << 4) + (m & 15) : m;
+    const int mr = ar & 7;                           // row inside its 8-row atom
     const bool issuer = q == 0 && lane == 0;         // packed-weight TMA
     const bool sc_issuer = issuer && grp == 0;       // tile-scale copies
     uint64_t* wf = w_full + grp * WG;
@@ -363,11 +380,11 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     const uint32_t nh = total > grp ? (total - grp + 1) / 2 : 0;  // this group's stages
     // first weight row (e * N + n0) of local tile tl
     auto tile_row = [&](int64_t tl) -> int64_t {
-      const TileInfo ti = tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E, BT);
+      const TileInfo ti = tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E, BT, NS);
       return (int64_t)ti.e * N + ti.n0;
     };
     auto tile_n0 = [&](int64_t tl) -> int32_t {
-      return tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E, BT).n0;
+      return tile_info(blockIdx.x + tl * gridDim.x, off_s, ts_s, E, BT, NS).n0;
     };
     // cursor: local tile tl and stage kb of group stage h; step() = h + 1
     struct Cursor {
@@ -392,7 +409,13 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       const uint32_t slot = issued % WG;
       ++issued;
       mbar_arrive_expect_tx(&wf[slot], kWStageBytes);
-      tma_load_2d(wring + slot * kWStageBytes, &tmw, wc.kb * (BK / 2), wrow0, &wf[slot]);
+      if (kGLU) {  // 64 gate rows, then the matching 64 up rows
+        tma_load_2d(wring + slot * kWStageBytes, &tmw64, wc.kb * (BK / 2), wrow0, &wf[slot]);
+        tma_load_2d(wring + slot * kWStageBytes + kWStageBytes / 2, &tmw64, wc.kb * (BK / 2),
+                    wrow0 + glu_i, &wf[slot]);
+      } else {
+        tma_load_2d(wring + slot * kWStageBytes, &tmw, wc.kb * (BK / 2), wrow0, &wf[slot]);
+      }
       if (step(wc) && issued < nh) wrow0 = (int32_t)tile_row(wc.tl);
     };
     // one tile's scales: rows e*N + n0 .. +127 (clipped at the end of the
@@ -401,12 +424,20 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     int64_t sc_issued = 0;
     auto issue_sc = [&](int64_t tl) {
       const int64_t row0 = tile_row(tl);
-      const int64_t rows = min((int64_t)BM, total_rows - row0);
-      const uint32_t bytes = (uint32_t)(rows * srow);
       sc_issued = tl + 1;
-      mbar_arrive_expect_tx(&sc_full[tl & 1], bytes);
-      bulk_load(smem + Smem::sc + (tl & 1) * kScaleBuf,
-                reinterpret_cast<const uint8_t*>(pb.scale) + row0 * srow, bytes, &sc_full[tl & 1]);
+      const uint8_t* sbase = reinterpret_cast<const uint8_t*>(pb.scale);
+      uint8_t* sdst = smem + Smem::sc + (tl & 1) * kScaleBuf;
+      if (kGLU) {  // the gate rows' scales, then the up rows'
+        const uint32_t half = (uint32_t)(64 * srow);
+        mbar_arrive_expect_tx(&sc_full[tl & 1], 2 * half);
+        bulk_load(sdst, sbase + row0 * srow, half, &sc_full[tl & 1]);
+        bulk_load(sdst + half, sbase + (row0 + glu_i) * srow, half, &sc_full[tl & 1]);
+      } else {
+        const int64_t rows = min((int64_t)BM, total_rows - row0);
+        const uint32_t bytes = (uint32_t)(rows * srow);
+        mbar_arrive_expect_tx(&sc_full[tl & 1], bytes);
+        bulk_load(sdst, sbase + row0 * srow, bytes, &sc_full[tl & 1]);
+      }
     };
     // per-thread scale loads (when tile scales do not fit): cursor two
     // stages ahead of the decode and this thread's scale row of its tile
@@ -414,6 +445,9 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     const uint8_t* lrow = nullptr;  // scale row of weight row m, or null past N
     const int sbytes = F == Fmt::NF4 ? 4 : 2;  // scale bytes per stage
     auto lrow_of = [&](int64_t tl) -> const uint8_t* {
+      if (kGLU)  // gate row n0 + m, or up row glu_i + n0 + m - 64
+        return reinterpret_cast<const uint8_t*>(pb.scale) +
+               (tile_row(tl) + (m < 64 ? m : glu_i + m - 64)) * (int64_t)srow;
       const int32_t n0 = tile_n0(tl);
       if (n0 + m >= N) return nullptr;
       return reinterpret_cast<const uint8_t*>(pb.scale) + (tile_row(tl) + m) * (int64_t)srow;
@@ -505,7 +539,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       if (!__all_sync(0xffffffffu, good)) return false;
       if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], aph ^ 1u, abort, pb.err))) return false;
       // row m of the K-major, 128B-swizzled A tile: chunk c at (c ^ (m % 8))
-      uint8_t* dst = smem + Smem::a + as * kAStageBytes + m * 128;
+      uint8_t* dst = smem + Smem::a + as * kAStageBytes + ar * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(dst + ((c ^ mr) << 4)) =
@@ -549,7 +583,7 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
     AccSched acc;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      const TileInfo ti = tile_info(t, off_s, ts_s, E, BT);
+      const TileInfo ti = tile_info(t, off_s, ts_s, E, BT, NS);
       const bool wide = ti.nv > BH;
       const int ncol0 = ti.n0 + (int)q * 32;  // first output column of this warp
       const int sub = lane & 3;               // 16-byte piece of a row
@@ -571,6 +605,39 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[hf]);
           }
+          if (kGLU) {
+            // lane l holds A-tile row 32q + l: gate (l < 16) or up (l >= 16)
+            // of h column n0 + 16q + l % 16, for the chunk's 32 routed rows.
+            // The two lanes of a column split the rows: the gate lane takes
+            // rows 0-15, the up lane rows 16-31, each receiving the other
+            // operand by one shuffle.  Both operands are rounded to bf16
+            // (the gate_up output); h = bf16(silu(gate) * up) goes into a
+            // 32-row x 16-column transpose.
+            const bool glane = lane < 16;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float mine = __bfloat162float(
+                  __float2bfloat16_rn(__uint_as_float(glane ? r[j] : r[j + 16])));
+              const float send = __bfloat162float(
+                  __float2bfloat16_rn(__uint_as_float(glane ? r[j + 16] : r[j])));
+              const float other = __shfl_xor_sync(0xffffffffu, send, 16);
+              const float g = glane ? mine : other, u = glane ? other : mine;
+              *reinterpret_cast<uint16_t*>(stage + (glane ? j : j + 16) * 32 + (lane & 15) * 2) =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u));
+            }
+            __syncwarp();
+            // two lanes write one routed row's 32 bytes of h
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const int rr = (lane >> 1) + 16 * v;  // row within the chunk
+              const int row = c * 32 + rr;
+              if (row < rows)
+                *reinterpret_cast<uint4*>(pb.out + (int64_t)(ti.p0 + row0 + row) * ON + ti.n0 +
+                                          (int)q * 16 + (lane & 1) * 8) =
+                    *reinterpret_cast<const uint4*>(stage + rr * 32 + (lane & 1) * 16);
+            }
+            __syncwarp();
+          } else {
           // thread = output column ncol0 + lane, r[j] = routed row c*32 + j
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -584,10 +651,11 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
             const int rr = (lane >> 2) + 8 * v;  // row within the chunk
             const int row = c * 32 + rr;         // routed row within the half
             if (row < rows && subok)
-              *reinterpret_cast<uint4*>(pb.out + (int64_t)(ti.p0 + row0 + row) * N + ncol0 + sub * 8) =
+              *reinterpret_cast<uint4*>(pb.out + (int64_t)(ti.p0 + row0 + row) * ON + ncol0 + sub * 8) =
                   *reinterpret_cast<const uint4*>(stage + rr * kEpiRowBytes + sub * 16);
           }
           __syncwarp();
+          }
         }
       }
       acc.next(wide);
@@ -648,7 +716,7 @@ size_t gemm_smem_bytes(int32_t E) {
 }
 
 cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
-                        cudaStream_t s) {
+                        cudaStream_t s, int64_t glu_i) {
   if (pb.P == 0 || pb.N == 0) return cudaSuccess;
   CUtensorMap tmx;
   // identity rows: boxes of 64 K x 256 rows (one per tile half); gathered rows use cp.async and
@@ -663,31 +731,46 @@ cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
                   (uint64_t)pb.K * 2, BK, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   // packed weights [E*N rows, K/2 bytes]: boxes of 32 bytes (one 64-K stage)
-  // x 128 rows; rows past E*N read as zeros
-  CUtensorMap tmw;
+  // x 128 rows (x 64 rows for the SwiGLU tiles' gate and up halves); rows
+  // past E*N read as zeros
+  CUtensorMap tmw, tmw64;
   e = make_map_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.w, (uint64_t)pb.K / 2,
                   (uint64_t)pb.E * (uint64_t)pb.N, (uint64_t)pb.K / 2, BK / 2, BM,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
   if (e != cudaSuccess) return e;
-  // A tile's scales (128 rows x srow bytes, contiguous) come by one bulk
-  // copy when they fit the buffer, there are at least two stages per tile
-  // (so both decode groups take part in every tile) and every copy stays
-  // 16-byte aligned: rows start at multiples of 128, so N * srow and the
-  // array's address must be multiples of 16.
+  e = make_map_2d(&tmw64, CU_TENSOR_MAP_DATA_TYPE_UINT8, pb.w, (uint64_t)pb.K / 2,
+                  (uint64_t)pb.E * (uint64_t)pb.N, (uint64_t)pb.K / 2, BK / 2, 64,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (e != cudaSuccess) return e;
+  // A tile's scales (128 rows x srow bytes, contiguous; for SwiGLU tiles two
+  // ranges of 64 rows) come by bulk copy when they fit the buffer, there are
+  // at least two stages per tile (so both decode groups take part in every
+  // tile) and every copy stays 16-byte aligned: rows start at multiples of
+  // 64, so N * srow, glu_i * srow and the array's address must be multiples
+  // of 16.
   const int srow = (f == Fmt::NF4) ? (int)(pb.K / 64) * 4 : (int)(pb.K / 32);
   const int tile_scales = (pb.K / BK >= 2) && (BM * srow <= kScaleBuf) &&
-                          ((pb.N * srow) % 16 == 0) &&
+                          ((pb.N * srow) % 16 == 0) && ((64 * (int64_t)srow) % 16 == 0) &&
+                          ((glu_i * srow) % 16 == 0) &&
                           (reinterpret_cast<uintptr_t>(pb.scale) % 16 == 0);
   const size_t smem = gemm_smem_bytes(pb.E);
   // wide tiles when activations come by TMA (identity rows), narrow when
   // they are gathered through row_to_token
   const bool wide = pb.row_to_token == nullptr;
-  auto k = (f == Fmt::NF4) ? (wide ? gemm_kernel<Fmt::NF4, true> : gemm_kernel<Fmt::NF4, false>)
-                           : (wide ? gemm_kernel<Fmt::MXFP4, true> : gemm_kernel<Fmt::MXFP4, false>);
+  const bool glu = glu_i > 0;
+  using KFn = void (*)(const GroupedProblem, const CUtensorMap, const CUtensorMap,
+                       const CUtensorMap, const CUtensorMap, const int, const int, const int32_t);
+  KFn k;
+#define GBW_GEMM_PICK(FF)                                                              \
+  k = glu ? (wide ? gemm_kernel<FF, true, true> : gemm_kernel<FF, false, true>)        \
+          : (wide ? gemm_kernel<FF, true, false> : gemm_kernel<FF, false, false>);
+  if (f == Fmt::NF4) { GBW_GEMM_PICK(Fmt::NF4) } else { GBW_GEMM_PICK(Fmt::MXFP4) }
+#undef GBW_GEMM_PICK
   e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<num_sms, kThreads, smem, s>>>(pb, tmx, tmx32, tmw, srow, tile_scales);
+  k<<<num_sms, kThreads, smem, s>>>(pb, tmx, tmx32, tmw, tmw64, srow, tile_scales,
+                                     (int32_t)glu_i);
   return cudaGetLastError();
 }
 

@@ -32,6 +32,12 @@
 //          G lanes of a row reduce with shuffles, two rows at a time (the
 //          lanes first swap halves, so a pair costs one shuffle more than a
 //          single row).
+// SwiGLU variant (the gate_up projection of the fused expert pass at decode
+// sizes, G = 32): virtual row 2j of a routed row is gate row j and 2j + 1 is
+// up row I + j, so a round's groups pair up; the pair reduction leaves the
+// gate total in the lower half of the lanes and the up total in the upper
+// half, and one more shuffle lets lane 0 write h = bf16(silu(bf16 gate) *
+// bf16 up) to h [P, I].
 // Numerics: MXFP4 codes are exact in bf16, so the products are exact.  NF4
 // codebook values are rounded to bf16 once (relative error <= 2^-9), and
 // the absmax multiplies the partial sum in fp32; the result stays well
@@ -132,12 +138,14 @@ struct Round {
 };
 
 // The row groups [g0, g1) of one warp, after the kernel's prologue.
-template <Fmt F, int G, int UPL, uint32_t kBase>
+template <Fmt F, int G, int UPL, bool kGLU, uint32_t kBase>
 __device__ __forceinline__ void gemv_main(const GroupedProblem& pb, const int32_t* off_s,
                                           int64_t g0, int64_t g1, int npass, int32_t tok,
                                           uint32_t base, bool waited) {
+  static_assert(!kGLU || G == 32, "the SwiGLU variant takes one row per group");
   constexpr int RG = 32 / G;                // rows per row group
-  constexpr int MG = Round<UPL>::MG;        // row groups per load round
+  // row groups per load round (even for SwiGLU: gate/up pairs)
+  constexpr int MG = kGLU ? (Round<UPL>::MG & ~1) : Round<UPL>::MG;
   const int lane = threadIdx.x & 31;
   const int li = lane % G, rs = lane / G;
   const int64_t K = pb.K, N = pb.N;
@@ -161,9 +169,13 @@ __device__ __forceinline__ void gemv_main(const GroupedProblem& pb, const int32_
     // one round: up to MG row groups of one routed row (one x)
     int cnt = (int)min((int64_t)MG, g1 - g);
     cnt = (int)min((int64_t)cnt, (N - n) / RG);
-    const int64_t wrow0 = (int64_t)e * N + n + rs;  // weight row of group 0
+    // weight row of group 0; SwiGLU: gate rows from wp, up rows from wpu
+    // (group k is gate or up row (n + k) / 2)
+    const int64_t I = N / 2;
+    const int64_t wrow0 = kGLU ? (int64_t)e * N + n / 2 : (int64_t)e * N + n + rs;
     const uint4* const wp = w16 + wrow0 * U;
-    const int64_t s0 = wrow0 * srow;
+    const uint4* const wpu = w16 + (wrow0 + I) * U;
+    const int64_t s0 = wrow0 * srow, s0u = (wrow0 + I) * srow;
     float acc[MG];
 #pragma unroll
     for (int k = 0; k < MG; ++k) acc[k] = 0.0f;
@@ -180,11 +192,13 @@ __device__ __forceinline__ void gemv_main(const GroupedProblem& pb, const int32_
           q[k][i] = make_uint4(0u, 0u, 0u, 0u);
           sc[k][i] = 0u;
           if (k < cnt && uo[i] < U) {
-            q[k][i] = __ldg(wp + k * wstride + uo[i]);
+            const uint4* rp = kGLU ? ((k & 1) ? wpu : wp) + (int64_t)(k >> 1) * U : wp + k * wstride;
+            const int64_t so = kGLU ? ((k & 1) ? s0u : s0) + (int64_t)(k >> 1) * srow : s0 + k * sstride;
+            q[k][i] = __ldg(rp + uo[i]);
             if (F == Fmt::NF4)
-              sc[k][i] = __ldg(reinterpret_cast<const uint32_t*>(pb.scale) + s0 + k * sstride + (uo[i] >> 1));
+              sc[k][i] = __ldg(reinterpret_cast<const uint32_t*>(pb.scale) + so + (uo[i] >> 1));
             else
-              sc[k][i] = __ldg(reinterpret_cast<const uint8_t*>(pb.scale) + s0 + k * sstride + uo[i]);
+              sc[k][i] = __ldg(reinterpret_cast<const uint8_t*>(pb.scale) + so + uo[i]);
           }
         }
       if ((int64_t)tok * npass + pass != xkey) {
@@ -228,10 +242,19 @@ __device__ __forceinline__ void gemv_main(const GroupedProblem& pb, const int32_
         keep += __shfl_xor_sync(0xffffffffu, hi ? a0 : a1, G / 2, G);
 #pragma unroll
         for (int o = G / 4; o; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o, G);
-        const int k = 2 * m + (hi ? 1 : 0);
-        if ((li & (G / 2 - 1)) == 0 && k < cnt)
-          pb.out[(int64_t)p * N + n + (int64_t)k * RG + rs] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(keep));
+        if (kGLU) {
+          // lower half: gate total of h column (n / 2 + m); upper half: up
+          const float g = __bfloat162float(__float2bfloat16_rn(keep));
+          const float u = __shfl_xor_sync(0xffffffffu, g, G / 2);
+          if (lane == 0)
+            pb.out[(int64_t)p * I + n / 2 + m] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.0f + expf(-g)) * u));
+        } else {
+          const int k = 2 * m + (hi ? 1 : 0);
+          if ((li & (G / 2 - 1)) == 0 && k < cnt)
+            pb.out[(int64_t)p * N + n + (int64_t)k * RG + rs] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(keep));
+        }
       }
     }
     // advance
@@ -250,7 +273,7 @@ __device__ __forceinline__ void gemv_main(const GroupedProblem& pb, const int32_
   }
 }
 
-template <Fmt F, int G, int UPL>
+template <Fmt F, int G, int UPL, bool kGLU>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -260,10 +283,13 @@ gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
   const int warp = threadIdx.x >> 5;
 
   // this warp's row groups: a contiguous chunk of the CTA's contiguous range
-  const int64_t c0 = ngroups * blockIdx.x / gridDim.x;
-  const int64_t c1 = ngroups * (blockIdx.x + 1) / gridDim.x;
-  const int64_t g0 = c0 + (c1 - c0) * warp / kWarps;
-  const int64_t g1 = c0 + (c1 - c0) * (warp + 1) / kWarps;
+  // (in gate/up pairs for SwiGLU)
+  constexpr int64_t A = kGLU ? 2 : 1;
+  const int64_t na = ngroups / A;
+  const int64_t c0 = na * blockIdx.x / gridDim.x;
+  const int64_t c1 = na * (blockIdx.x + 1) / gridDim.x;
+  const int64_t g0 = A * (c0 + (c1 - c0) * warp / kWarps);
+  const int64_t g1 = A * (c0 + (c1 - c0) * (warp + 1) / kWarps);
 
   // Programmatic dependent launch.  Without GBW_FLAG_OVERLAP_PREV every
   // input may come from the kernel launched just before this one, so this
@@ -307,9 +333,9 @@ gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
     return;
   }
   if (base == kLutBaseGuess)
-    gemv_main<F, G, UPL, kLutBaseGuess>(pb, off_s, g0, g1, npass, tok0, base, !early);
+    gemv_main<F, G, UPL, kGLU, kLutBaseGuess>(pb, off_s, g0, g1, npass, tok0, base, !early);
   else
-    gemv_main<F, G, UPL, kRuntimeBase>(pb, off_s, g0, g1, npass, tok0, base, !early);
+    gemv_main<F, G, UPL, kGLU, kRuntimeBase>(pb, off_s, g0, g1, npass, tok0, base, !early);
 }
 
 struct Shape {
@@ -334,10 +360,10 @@ Shape pick_shape(int64_t U) {
 // Dynamic shared memory: the 64 KB table, then the offsets.
 size_t gemv_smem(int32_t E) { return (size_t)kLutBytes + 4 * (size_t)(E + 1); }
 
-template <Fmt F, int G, int UPL>
+template <Fmt F, int G, int UPL, bool kGLU = false>
 cudaError_t launch_t(const GroupedProblem& pb, int64_t ngroups, int npass,
                      int grid, cudaStream_t s) {
-  auto k = gemv_kernel<F, G, UPL>;
+  auto k = gemv_kernel<F, G, UPL, kGLU>;
   const size_t smem = gemv_smem(pb.E);
   // the shared-memory opt-in is set once per device and size
   static size_t opted[64];
@@ -382,11 +408,26 @@ bool gemv_fits(Fmt, const GroupedProblem& pb, int) {
 }
 
 cudaError_t launch_gemv(Fmt f, const GroupedProblem& pb, int num_sms,
-                        cudaStream_t s) {
+                        cudaStream_t s, bool glu) {
   if (pb.P == 0 || pb.N == 0) return cudaSuccess;
-  const Shape sh = pick_shape(pb.K / 32);
+  const int64_t U = pb.K / 32;
+  // SwiGLU: one row per group (G = 32), as many units per lane as the row needs
+  const Shape sh = glu ? Shape{32, (int)std::min<int64_t>(3, (U + 31) / 32), (int)((U + 95) / 96)}
+                       : pick_shape(U);
   const int64_t ngroups = pb.P * (pb.N / (32 / sh.G));
-  const int grid = (int)std::min<int64_t>(num_sms, (ngroups + kWarps - 1) / kWarps);
+  // the kernel keys its activation rows as token * npass + pass in 32 bits
+  if ((int64_t)std::max<int64_t>(pb.T, pb.P) * sh.npass >= INT32_MAX) return cudaErrorInvalidValue;
+  const int grid = (int)std::min<int64_t>(num_sms, (ngroups / (glu ? 2 : 1) + kWarps - 1) / kWarps);
+  if (glu) {
+#define GBW_GEMV_GLU(FF)                                                              \
+  switch (sh.UPL) {                                                                   \
+    case 1: return launch_t<FF, 32, 1, true>(pb, ngroups, sh.npass, grid, s);         \
+    case 2: return launch_t<FF, 32, 2, true>(pb, ngroups, sh.npass, grid, s);         \
+    default: return launch_t<FF, 32, 3, true>(pb, ngroups, sh.npass, grid, s);        \
+  }
+    if (f == Fmt::NF4) { GBW_GEMV_GLU(Fmt::NF4) } else { GBW_GEMV_GLU(Fmt::MXFP4) }
+#undef GBW_GEMV_GLU
+  }
   return f == Fmt::NF4 ? launch_f<Fmt::NF4>(pb, sh, ngroups, grid, s)
                        : launch_f<Fmt::MXFP4>(pb, sh, ngroups, grid, s);
 }

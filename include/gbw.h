@@ -141,6 +141,48 @@ GBW_API gbw_status gmxfp4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N
                                 const int32_t* expert_offsets, uint16_t* dx,
                                 void* stream);
 
+/* Fused expert pass, NF4 ("Receipts-driven engineering", "The numbers":
+ * the fused training row over all 48 Qwen3-30B-A3B layers -- the expert
+ * MLP runs gate_up, the SwiGLU combine and down in one pass per routed row).
+ *   gate_up[p, :] = x[tok(p)] @ Wgu_e(p)^T          (2I columns, bf16)
+ *   h[p, j]       = bf16( silu(gate_up[p, j]) * gate_up[p, I + j] ),
+ *                   silu(v) = v / (1 + e^-v), evaluated in fp32
+ *   out[p, :]     = h[p] @ Wdn_e(p)^T                (H columns, bf16)
+ * The page names the pass but prints neither the activation nor the
+ * gate/up layout; the reading taken is the standard SwiGLU with the gate
+ * rows [0, I) stacked above the up rows [I, 2I) of each expert's gate_up
+ * weight.
+ *   x          [T, H] bf16 row-major; row_to_token / expert_offsets / P as
+ *              in gnf4_grouped_gemm
+ *   gu_packed  [E, 2I, H/2] uint8, gu_absmax [E, 2I, H/64] fp32
+ *   dn_packed  [E, H, I/2] uint8, dn_absmax [E, H, I/64] fp32
+ *   h          [P, I] bf16 WORKSPACE supplied by the caller: written by the
+ *              gate_up kernel, read by the down kernel (it keeps h)
+ *   out        [P, H] bf16, expert-sorted row order
+ *   mode       AUTO: both projections on the bandwidth GEMV when P <= 8,
+ *              else both on the tensor cores; GEMM / GEMV force a path.  No
+ *              flags.  SwiGLU is computed where the gate and up sums meet
+ *              (the GEMM epilogue pairs them in one tile, the GEMV in one
+ *              warp), so gate_up is never written out.
+ * Requires H % 64 == 0, I % 64 == 0, 16-byte aligned x, weights, h and out.
+ * Two kernels are launched on `stream`, in order. */
+GBW_API gbw_status gnf4_grouped_expert_mlp(const uint16_t* x, int64_t T, int64_t H,
+                                   const uint8_t* gu_packed, const float* gu_absmax,
+                                   const uint8_t* dn_packed, const float* dn_absmax,
+                                   int32_t E, int64_t I, const int32_t* expert_offsets,
+                                   const int32_t* row_to_token, int64_t P, uint16_t* h,
+                                   uint16_t* out, int32_t mode, void* stream);
+
+/* Fused expert pass, MXFP4 (gate_up blocks [E, 2I, H/32, 16] + scales
+ * [E, 2I, H/32]; down blocks [E, H, I/32, 16] + scales [E, H, I/32], e8m0,
+ * 2-byte aligned).  Everything else as gnf4_grouped_expert_mlp. */
+GBW_API gbw_status gmxfp4_grouped_expert_mlp(const uint16_t* x, int64_t T, int64_t H,
+                                     const uint8_t* gu_blocks, const uint8_t* gu_scales,
+                                     const uint8_t* dn_blocks, const uint8_t* dn_scales,
+                                     int32_t E, int64_t I, const int32_t* expert_offsets,
+                                     const int32_t* row_to_token, int64_t P, uint16_t* h,
+                                     uint16_t* out, int32_t mode, void* stream);
+
 /* Decode packed weights to bf16 ("grouped-nf4-gemm 0.43.0", "Try the
  * packers and byte checks on CPU", example 1: dequant_ref).  Bit-exact:
  * w[r, k] = bf16_rn(fp32(NF4[q] * absmax[r, k/64])).  rows counts all

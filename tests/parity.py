@@ -61,3 +61,34 @@ def assert_rows_exact_operands(gpu_bf16_bits, oracle_f64, rel_acc=1e-4, what="")
     ratio = float(np.max(err / bound))
     assert np.all(err <= bound), f"{what}: worst |err|/bound = {ratio:.3g}"
     return ratio
+
+
+def swiglu_tolerance(gu_bf16_bits, rel: float = 1e-2) -> np.ndarray:
+    """Per-element tolerance of h = bf16(silu(gate) * up) computed from a
+    gate_up output that is itself only fixed within the matmul tolerance:
+    that tolerance (rel * rms(gate_up row) + 1 ulp, which also covers a bf16
+    rounding of gate or up that lands one ulp away) propagated through
+    silu(g) * u to second order, plus one bf16 ulp of h.  gu [P, 2I] holds the
+    oracle's gate (columns [0, I)) and up ([I, 2I)) values."""
+    gu = bf16_bits_to_f64(gu_bf16_bits)
+    tol = row_tolerance(gu, rel)
+    I = gu.shape[-1] // 2
+    g, u, tg, tu = gu[..., :I], gu[..., I:], tol[..., :I], tol[..., I:]
+    sig = 1.0 / (1.0 + np.exp(-g))
+    silu = g * sig
+    dsilu = sig * (1.0 + g * (1.0 - sig))
+    # first order, plus the second-order terms (cross term silu'(g) dg du and
+    # the curvature of silu, |silu''| <= 1/2) that matter near g, u ~ 0
+    return (np.abs(dsilu * u) * tg + np.abs(silu) * tu + np.abs(dsilu) * tg * tu
+            + 0.25 * tg * tg * (np.abs(u) + tu) + bf16_ulp(silu * u))
+
+
+def assert_close_to(gpu_bf16_bits, oracle_f64, tol, what=""):
+    """|gpu - oracle| <= tol elementwise (a non-empty comparison)."""
+    g = bf16_bits_to_f64(gpu_bf16_bits)
+    o = np.asarray(oracle_f64, np.float64)
+    assert g.shape == o.shape and o.size > 0, (g.shape, o.shape)
+    err = np.abs(g - o)
+    worst = float(np.max(err / tol))
+    assert np.all(err <= tol), f"{what}: {o.size} elements, worst |err|/tol = {worst:.3g}"
+    return worst

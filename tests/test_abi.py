@@ -17,8 +17,8 @@ def _declared():
 def test_header_declares_the_entry_points():
     names = set(_declared())
     for n in ["gnf4_grouped_gemm", "gmxfp4_grouped_gemm", "gnf4_grouped_dgrad",
-              "gmxfp4_grouped_dgrad",
-              "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
+              "gmxfp4_grouped_dgrad", "gnf4_grouped_expert_mlp",
+              "gmxfp4_grouped_expert_mlp", "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
               "gmxfp4_quantize", "gbw_device_status", "gbw_status_string",
               "gbw_version"]:
         assert n in names, n
@@ -87,3 +87,27 @@ def test_dgrad_and_codec_validation():
     assert L.gmxfp4_quantize(C.c_void_p(8), 4, 64, p, p, None) == 3
     assert L.gnf4_dequant(p, p, 4, 96, p, None) == 2
     assert b"K % 64" in L.gbw_status_string(2)  # text of the last error
+
+
+@pytest.mark.parametrize("fn", ["gnf4_grouped_expert_mlp", "gmxfp4_grouped_expert_mlp"])
+def test_fused_pass_host_validation(fn):
+    import grouped_bit_weight_b200 as gbw
+    f = getattr(gbw.lib, fn)
+    SHAPE, NULL, ALIGN = 2, 1, 3
+
+    def call(**kw):
+        a = dict(x=16, T=8, H=256, gu=16, gs=16, dn=16, ds=16, E=2, I=128, off=16,
+                 r2t=None, P=8, h=16, out=16, mode=0)
+        a.update(kw)
+        v = lambda k: None if a[k] is None else C.c_void_p(a[k])
+        return f(v("x"), a["T"], a["H"], v("gu"), v("gs"), v("dn"), v("ds"), a["E"], a["I"],
+                 v("off"), v("r2t"), a["P"], v("h"), v("out"), a["mode"], None)
+    assert call(H=320 + 32) == SHAPE      # H % 64
+    assert call(I=96) == SHAPE            # I % 64
+    assert call(E=0) == SHAPE
+    assert call(mode=0x100) == SHAPE      # no flags on the fused pass
+    assert call(T=4, P=8) == SHAPE        # identity rows need T >= P
+    assert call(h=0) == NULL
+    assert call(dn=0) == NULL
+    assert call(h=24) == ALIGN
+    assert call(gs=17) == ALIGN
