@@ -17,7 +17,8 @@ import torch
 __all__ = [
     "lib", "GbwError", "gnf4_grouped_gemm", "gmxfp4_grouped_gemm",
     "gnf4_grouped_dgrad", "gmxfp4_grouped_dgrad", "gnf4_grouped_expert_mlp",
-    "gmxfp4_grouped_expert_mlp", "gnf4_dequant", "gmxfp4_dequant", "gnf4_quantize",
+    "gmxfp4_grouped_expert_mlp", "gnf4_grouped_expert_mlp_noalloc", "gnf4_dequant",
+    "gmxfp4_dequant", "gnf4_quantize",
     "gmxfp4_quantize", "device_status", "MODE_AUTO", "MODE_GEMM", "MODE_GEMV",
     "DEVERR_OFFSETS", "DEVERR_TOKEN", "DEVERR_TIMEOUT", "FLAG_OVERLAP_PREV",
     "EXPORTS",
@@ -50,6 +51,7 @@ EXPORTS = {
     "gmxfp4_grouped_dgrad": (C.c_int, [_P, _I64, _I64, _P, _P, _I32, _I64, _P, _P, _P]),
     "gnf4_grouped_expert_mlp": (C.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _I32, _I64, _P, _P, _I64, _P, _P, _I32, _P]),
     "gmxfp4_grouped_expert_mlp": (C.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _I32, _I64, _P, _P, _I64, _P, _P, _I32, _P]),
+    "gnf4_grouped_expert_mlp_noalloc": (C.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _I32, _I64, _P, _P, _I64, _P, _I32, _P]),
     "gnf4_dequant": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "gmxfp4_dequant": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "gnf4_quantize": (C.c_int, [_P, _I64, _I64, _P, _P, _P]),
@@ -288,6 +290,40 @@ def gmxfp4_grouped_expert_mlp(x, gu_blocks, gu_scales, dn_blocks, dn_scales, exp
     return _expert_mlp(lib.gmxfp4_grouped_expert_mlp, "gmxfp4_grouped_expert_mlp", x, gu_blocks,
                        gu_scales, dn_blocks, dn_scales, torch.uint8, 32, expert_offsets,
                        row_to_token, h, out, mode)
+
+
+def gnf4_grouped_expert_mlp_noalloc(x, gu_packed, gu_absmax, dn_packed, dn_absmax,
+                                    expert_offsets, row_to_token=None, out=None, mode="auto"):
+    """gnf4_grouped_expert_mlp for callers that cannot supply device memory
+    for h: the library keeps h in its own fixed 4 MiB array (P * I <=
+    2,097,152).  Calls that may overlap on the GPU share that array and must
+    be ordered.  Returns out [P, H] (allocated here when not given; pass
+    `out` to allocate nothing at all)."""
+    where = "gnf4_grouped_expert_mlp_noalloc"
+    _need(x, "x", torch.bfloat16)
+    _need(expert_offsets, "expert_offsets", torch.int32)
+    T, H = x.shape
+    E, I = gu_packed.shape[0], gu_packed.shape[1] // 2
+    _numel(gu_packed, "gate_up weights", E * 2 * I * (H // 2), where)
+    _numel(gu_absmax, "gate_up scales", E * 2 * I * (H // 64), where)
+    _numel(dn_packed, "down weights", E * H * (I // 2), where)
+    _numel(dn_absmax, "down scales", E * H * (I // 64), where)
+    _numel(expert_offsets, "expert_offsets", E + 1, where)
+    P = row_to_token.numel() if row_to_token is not None else T
+    if out is not None:
+        _need(out, "out", torch.bfloat16)
+        if tuple(out.shape) != (P, H):
+            raise ValueError(f"{where}: out must be [{P}, {H}]")
+    dev = _on_device(where, x=x, gu=gu_packed, gs=gu_absmax, dn=dn_packed, ds=dn_absmax,
+                     expert_offsets=expert_offsets, row_to_token=row_to_token, out=out)
+    if out is None:
+        out = torch.empty((P, H), dtype=torch.bfloat16, device=dev)
+    m = _MODES[mode] if isinstance(mode, str) else int(mode)
+    with torch.cuda.device(dev):
+        _check(lib.gnf4_grouped_expert_mlp_noalloc(
+            _ptr(x), T, H, _ptr(gu_packed), _ptr(gu_absmax), _ptr(dn_packed), _ptr(dn_absmax),
+            E, I, _ptr(expert_offsets), _ptr(row_to_token), P, _ptr(out), m, _stream(dev)), where)
+    return out
 
 
 def _dequant(fn, where, w, scale, scale_dtype, K, sdiv, out_shape, out):

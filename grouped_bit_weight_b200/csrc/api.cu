@@ -278,6 +278,57 @@ gbw_status gmxfp4_grouped_expert_mlp(const uint16_t* x, int64_t T, int64_t H,
                     expert_offsets, row_to_token, P, h, out, mode, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Fused expert pass without any device allocation.
+//
+// gnf4_grouped_expert_mlp asks the caller for the h workspace.  Some callers
+// cannot provide one: a plugin inside an inference engine whose device memory
+// is already handed out by the engine, or a serving loop that forbids device
+// allocation after warm-up because cudaMalloc can synchronise the device and
+// fragments memory a caching allocator holds.  For them the h rows live in a
+// fixed array in this library's device image.  Every device that loads the
+// library holds the array until the process exits, so it is kept small.
+// ---------------------------------------------------------------------------
+
+// h scratch of gnf4_grouped_expert_mlp_noalloc: P * I bf16 values at most.
+constexpr int64_t kNoAllocHElems = (int64_t)1 << 21;  // 2,097,152 values, 4 MiB
+static __device__ __align__(256) uint16_t g_noalloc_h[kNoAllocHElems];
+
+// Device address of g_noalloc_h per device.  In host code the name
+// g_noalloc_h is only a host-side stand-in, so the address is looked up once
+// per device, with that device current, on the first call there.
+static uint16_t* g_noalloc_ptr[kMaxDevices];
+static cudaError_t g_noalloc_err[kMaxDevices];
+static std::once_flag g_noalloc_once[kMaxDevices];
+
+gbw_status gnf4_grouped_expert_mlp_noalloc(const uint16_t* x, int64_t T, int64_t H,
+                                           const uint8_t* gu_packed, const float* gu_absmax,
+                                           const uint8_t* dn_packed, const float* dn_absmax,
+                                           int32_t E, int64_t I, const int32_t* expert_offsets,
+                                           const int32_t* row_to_token, int64_t P,
+                                           uint16_t* out, int32_t mode, void* stream) {
+  if (P > 0 && I > 0 && P <= INT32_MAX && I <= ((int64_t)1 << 29) && P * I > kNoAllocHElems) {
+    snprintf(g_msg, sizeof(g_msg),
+             "P * I = %lld exceeds the %lld bf16 values of the no-allocation h scratch",
+             (long long)(P * I), (long long)kNoAllocHElems);
+    return GBW_ERR_SHAPE;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return launch_error(e);
+  if (dev < 0 || dev >= kMaxDevices) return GBW_ERR_ARCH;
+  std::call_once(g_noalloc_once[dev], [dev]() {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_h);
+    g_noalloc_ptr[dev] = static_cast<uint16_t*>(p);
+  });
+  if (g_noalloc_err[dev] != cudaSuccess) return launch_error(g_noalloc_err[dev]);
+  // every h element the down projection reads is written by gate_up in the
+  // same call, so the array's previous contents never matter
+  return expert_mlp(Fmt::NF4, x, T, H, gu_packed, gu_absmax, dn_packed, dn_absmax, E, I,
+                    expert_offsets, row_to_token, P, g_noalloc_ptr[dev], out, mode, stream);
+}
+
 gbw_status gnf4_dequant(const uint8_t* packed, const float* absmax,
                         int64_t rows, int64_t K, uint16_t* w_out,
                         void* stream) {

@@ -183,6 +183,31 @@ GBW_API gbw_status gmxfp4_grouped_expert_mlp(const uint16_t* x, int64_t T, int64
                                      const int32_t* row_to_token, int64_t P, uint16_t* h,
                                      uint16_t* out, int32_t mode, void* stream);
 
+/* Fused NF4 expert pass that allocates nothing and takes no workspace.
+ * This entry point has no counterpart on the source pages; it exists for
+ * callers that cannot hand the library device memory at call time -- for
+ * example a plugin running inside an inference engine that has already
+ * reserved all device memory for itself, or a serving loop that forbids
+ * allocation after warm-up (cudaMalloc may synchronise the device and
+ * fragment memory held by a caching allocator).
+ *   Same arguments and results as gnf4_grouped_expert_mlp, without h: the h
+ *   rows go to a fixed scratch array inside the library's device image
+ *   (4 MiB, which every device that loads the library keeps until the
+ *   process exits).
+ *   Limit: P * I <= 2,097,152; larger problems return GBW_ERR_SHAPE.
+ *   The first call on a device looks up the scratch address for that device
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   All calls share the one array: calls whose kernels may overlap on the
+ *   GPU (different streams, or several host threads) race on it and must be
+ *   ordered by the caller.  No call depends on what an earlier call left
+ *   there.  No device memory is allocated or freed. */
+GBW_API gbw_status gnf4_grouped_expert_mlp_noalloc(const uint16_t* x, int64_t T, int64_t H,
+                                           const uint8_t* gu_packed, const float* gu_absmax,
+                                           const uint8_t* dn_packed, const float* dn_absmax,
+                                           int32_t E, int64_t I, const int32_t* expert_offsets,
+                                           const int32_t* row_to_token, int64_t P,
+                                           uint16_t* out, int32_t mode, void* stream);
+
 /* Decode packed weights to bf16 ("grouped-nf4-gemm 0.43.0", "Try the
  * packers and byte checks on CPU", example 1: dequant_ref).  Bit-exact:
  * w[r, k] = bf16_rn(fp32(NF4[q] * absmax[r, k/64])).  rows counts all
