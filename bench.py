@@ -680,6 +680,37 @@ def run_case(args, dev):
         fn = lambda: gbw.gmxfp4_grouped_gemm(x, w[0], w[1], d_off, d_r2t, out=o)
         nbytes, unit = ((gemm_flops(P, L.N, L.K), "TFLOP/s") if T > 1
                         else (gemv_bytes("mxfp4", P, L.N, L.K, 1), "GB/s"))
+    elif c in ("mxfp4_dgrad_gate_up", "mxfp4_dgrad_down"):
+        L = synth.GPTOSS_GATE_UP if c.endswith("gate_up") else synth.GPTOSS_DOWN
+        w = make_mxfp4(torch, gbw, L.E, L.N, L.K, L.w_std, gen, dev)
+        off, _ = synth.uniform_routing(2048, L.E, 4, seed=7)
+        P = int(off[-1])
+        d_off = torch.from_numpy(off).to(dev)
+        dy = (torch.randn((P, L.N), generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
+        o = torch.empty((P, L.K), dtype=torch.bfloat16, device=dev)
+        fn = lambda: gbw.gmxfp4_grouped_dgrad(dy, w[0], w[1], d_off, out=o)
+        nbytes, unit = gemm_flops(P, L.N, L.K), "TFLOP/s"
+    elif c in ("fused_prefill", "fused_decode"):
+        GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
+        wgu = make_nf4(torch, gbw, GU.E, GU.N, GU.K, GU.w_std, gen, dev)
+        wdn = make_nf4(torch, gbw, DN.E, DN.N, DN.K, DN.w_std, gen, dev)
+        if c == "fused_prefill":
+            off, r2t = synth.prefill_routing()
+            T = 4096
+        else:
+            off, r2t = synth.decode_routing(GU.E, 8, 0)
+            T = 1
+        P = int(off[-1])
+        d_off, d_r2t = torch.from_numpy(off).to(dev), torch.from_numpy(r2t).to(dev)
+        x = torch.randn((T, GU.K), generator=gen, device=dev).to(torch.bfloat16)
+        h = torch.empty((P, DN.K), dtype=torch.bfloat16, device=dev)
+        o = torch.empty((P, DN.N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: gbw.gnf4_grouped_expert_mlp(x, wgu[0], wgu[1], wdn[0], wdn[1], d_off, d_r2t,
+                                                 h=h, out=o)
+        if T > 1:
+            nbytes, unit = gemm_flops(P, GU.N, GU.K) + gemm_flops(P, DN.N, DN.K), "TFLOP/s"
+        else:
+            nbytes, unit = gemv_bytes("nf4", 8, GU.N, GU.K, 1) + gemv_bytes("nf4", 8, DN.N, DN.K, 8), "GB/s"
     else:
         raise SystemExit(f"unknown case {c}")
     for _ in range(args.warmup):
