@@ -46,7 +46,7 @@ def bench_config(world):
     return {"workload": WORKLOAD, "weights": "nf4 (absmax fp32 per 64)",
             "activations": "bf16", "experts_cycled": f"{N_SETS} disjoint sets of 8",
             "l2": "inputs larger than L2: 340 MB of packed weights cycled, 21 MB per step",
-            "path": "bandwidth GEMV (GBW_MODE_AUTO picks it for P <= 8)",
+            "path": "bandwidth GEMV (GBW_MODE_AUTO picks it for P <= 4 E)",
             "parallelism": f"replicas x{world}"}
 
 
@@ -508,6 +508,27 @@ def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):
                          "SwiGLU then down, both on the bandwidth GEMV)",
                          gemv_bytes("nf4", 8, GU.N, GU.K, 1) + gemv_bytes("nf4", 8, DN.N, DN.K, 8), ms))
 
+    # a decode batch of 4 tokens (top-8: 32 routed rows, some experts with
+    # 2-3): AUTO takes the GEMV; an expert's rows are consecutive, so its
+    # weights come from HBM once and from L2 for its other rows.  bytes = the
+    # active experts' codes and scales once + x + out
+    bsets = [synth.uniform_routing(4, GU.E, 8, seed=200 + j) for j in range(N_SETS)]
+    boffs = [torch.from_numpy(a).to(dev) for a, _ in bsets]
+    br2ts = [torch.from_numpy(b).to(dev) for _, b in bsets]
+    xb = torch.randn((4, GU.K), generator=gen, device=dev).to(torch.bfloat16)
+    ob = torch.empty((32, GU.N), dtype=torch.bfloat16, device=dev)
+    it["j"] = 0
+
+    def batch_step():
+        j = it["j"] % N_SETS
+        it["j"] += 1
+        gbw.gnf4_grouped_gemm(xb, wgu[0], wgu[1], boffs[j], br2ts[j], out=ob, overlap_prev=True)
+    ms = graph_ms(batch_step, N_SETS)
+    act = float(np.mean([(np.diff(a) > 0).sum() for a, _ in bsets]))
+    nbytes = act * (GU.N * GU.K // 2 + GU.N * (GU.K // 64) * 4) + 4 * GU.K * 2 + 32 * GU.N * 2
+    out.append(hbm_entry(f"qwen3 decode batch of 4 tokens gate_up NF4 (32 routed rows over "
+                         f"{act:.1f} active experts; bytes count each expert's weights once)", nbytes, ms))
+
     # dequantise-then-GEMM comparator: decode the weights to bf16 in HBM
     # (the library's bit-exact decoder), then cuBLAS bf16 matmuls per expert
     out += dequant_comparator(torch, gbw, x, xd, wgu, wdn, off, r2t, d_r2t, sets, gu_prefill,
@@ -680,6 +701,21 @@ def run_case(args, dev):
         fn = lambda: gbw.gmxfp4_grouped_gemm(x, w[0], w[1], d_off, d_r2t, out=o)
         nbytes, unit = ((gemm_flops(P, L.N, L.K), "TFLOP/s") if T > 1
                         else (gemv_bytes("mxfp4", P, L.N, L.K, 1), "GB/s"))
+    elif c == "decode_batch4_gate_up":
+        L = synth.QWEN_GATE_UP
+        w = make_nf4(torch, gbw, L.E, L.N, L.K, L.w_std, gen, dev)
+        sets = [synth.uniform_routing(4, L.E, 8, seed=200 + j) for j in range(N_SETS)]
+        offs = [torch.from_numpy(o).to(dev) for o, _ in sets]
+        r2ts = [torch.from_numpy(r).to(dev) for _, r in sets]
+        x = torch.randn((4, L.K), generator=gen, device=dev).to(torch.bfloat16)
+        o = torch.empty((32, L.N), dtype=torch.bfloat16, device=dev)
+        it = {"i": 0}
+        def fn():
+            j = it["i"] % N_SETS
+            it["i"] += 1
+            gbw.gnf4_grouped_gemm(x, w[0], w[1], offs[j], r2ts[j], out=o)
+        act = float(np.mean([(np.diff(a) > 0).sum() for a, _ in sets]))
+        nbytes, unit = act * (L.N * L.K // 2 + L.N * (L.K // 64) * 4) + 4 * L.K * 2 + 32 * L.N * 2, "GB/s"
     elif c in ("mxfp4_dgrad_gate_up", "mxfp4_dgrad_down"):
         L = synth.GPTOSS_GATE_UP if c.endswith("gate_up") else synth.GPTOSS_DOWN
         w = make_mxfp4(torch, gbw, L.E, L.N, L.K, L.w_std, gen, dev)

@@ -277,7 +277,7 @@ def gnf4_grouped_expert_mlp(x, gu_packed, gu_absmax, dn_packed, dn_absmax, exper
     """Fused expert pass: gate_up [E, 2I, H/2] (gate rows then up rows),
     h = silu(gate) * up [P, I] (workspace, returned), down [E, H, I/2] ->
     out [P, H].  Returns (out, h).  mode "auto": both projections on the
-    bandwidth GEMV when P <= 8, else both on the tensor cores."""
+    bandwidth GEMV when P <= 4 * E, else both on the tensor cores."""
     return _expert_mlp(lib.gnf4_grouped_expert_mlp, "gnf4_grouped_expert_mlp", x, gu_packed,
                        gu_absmax, dn_packed, dn_absmax, torch.float32, 64, expert_offsets,
                        row_to_token, h, out, mode)

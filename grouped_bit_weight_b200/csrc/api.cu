@@ -135,8 +135,13 @@ gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
     return fail(GBW_ERR_SHAPE, "rows too long for the GEMV's shared-memory ring");
   if (!fits && K % 64)
     return fail(GBW_ERR_SHAPE, "rows too long for the GEMV and K % 64 != 0");
+  // AUTO: the bandwidth GEMV while experts average at most four routed rows
+  // (it streams each active expert's weights once and beats the tensor-core
+  // GEMM there: measured on B200 at Qwen3-30B-A3B shapes, the GEMM wins from
+  // about six rows per expert), and for K % 64 != 0, which the GEMM's 64-wide
+  // K stages do not take
   const bool gemv = mode == GBW_MODE_GEMV ||
-                    (mode == GBW_MODE_AUTO && fits && (P <= 8 || K % 64));
+                    (mode == GBW_MODE_AUTO && fits && (P <= 4 * (int64_t)E || K % 64));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = gemv ? launch_gemv(f, pb, sms, s) : launch_gemm(f, pb, sms, s);
   return e == cudaSuccess ? GBW_OK : launch_error(e);
@@ -249,7 +254,7 @@ static gbw_status expert_mlp(Fmt f, const uint16_t* x, int64_t T, int64_t H,
   // gate_up with SwiGLU fused into the output (h = silu(gate) * up), then
   // down over h (row p of h is routed row p); both on the bandwidth GEMV or
   // both on the tensor cores
-  const bool gemv = mode == GBW_MODE_GEMV || (mode == GBW_MODE_AUTO && P <= 8);
+  const bool gemv = mode == GBW_MODE_GEMV || (mode == GBW_MODE_AUTO && P <= 4 * (int64_t)E);
   GroupedProblem g{x, T, H, gu, gu_scale, E, 2 * I, offsets, row_to_token, P, h, err, 0};
   cudaError_t e = gemv ? launch_gemv(f, g, sms, s, true) : launch_gemm(f, g, sms, s, I);
   if (e != cudaSuccess) return launch_error(e);

@@ -52,7 +52,9 @@ typedef enum {
 } gbw_status;
 
 typedef enum {
-  GBW_MODE_AUTO = 0, /* GEMV when P <= 8, else the tensor-core GEMM */
+  GBW_MODE_AUTO = 0, /* GEMV when P <= 4 * E (at most ~4 routed rows per
+                        expert on average) or K % 64 != 0, else the
+                        tensor-core GEMM */
   GBW_MODE_GEMM = 1, /* force the tcgen05 grouped GEMM */
   GBW_MODE_GEMV = 2  /* force the bandwidth GEMV (no tensor cores) */
 } gbw_mode;
@@ -159,7 +161,7 @@ GBW_API gbw_status gmxfp4_grouped_dgrad(const uint16_t* dy, int64_t P, int64_t N
  *   h          [P, I] bf16 WORKSPACE supplied by the caller: written by the
  *              gate_up kernel, read by the down kernel (it keeps h)
  *   out        [P, H] bf16, expert-sorted row order
- *   mode       AUTO: both projections on the bandwidth GEMV when P <= 8,
+ *   mode       AUTO: both projections on the bandwidth GEMV when P <= 4 * E,
  *              else both on the tensor cores; GEMM / GEMV force a path.  No
  *              flags.  SwiGLU is computed where the gate and up sums meet
  *              (the GEMM epilogue pairs them in one tile, the GEMV in one

@@ -37,7 +37,7 @@ def _full_check(fmt, E, N, K, std, off, r2t, T, mode, seed=0, rel=1e-2):
     what = f"{fmt} {mode} E{E} N{N} K{K}"
     worst = assert_rows_close(got, ref, rel=rel, what=what)
     P = int(off[-1])
-    if mode == "gemm" or (mode == "auto" and P > 8):
+    if mode == "gemm" or (mode == "auto" and P > 4 * E and K % 64 == 0):
         assert_rows_exact_operands(got, ref, what=what)
     return worst
 
@@ -59,6 +59,32 @@ def test_qwen_decode(layer, mode):
     if T == 8:  # down projection: one distinct activation row per routed row
         r2t = None
     _full_check("nf4", layer.E, layer.N, layer.K, layer.w_std, off, r2t, T, mode)
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
+def test_gemv_experts_with_several_rows(fmt):
+    """Experts with 2-8 routed rows next to single-row and empty ones: the
+    GEMV reads each active expert's weights once and serves all its rows
+    (forced, and picked by AUTO since P <= 4 E)."""
+    E, N, K = 8, 512, 1024
+    counts = np.array([2, 8, 1, 1, 3, 0, 5, 1], np.int32)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    P = int(off[-1])
+    r2t = np.random.default_rng(90).integers(0, 12, P).astype(np.int32)
+    _full_check(fmt, E, N, K, 1.0, off, r2t, 12, "gemv", seed=91)
+    _full_check(fmt, E, N, K, 1.0, off, None, P, "auto", seed=92)
+
+
+@pytest.mark.parametrize("layer", [synth.QWEN_GATE_UP, synth.QWEN_DOWN])
+def test_qwen_decode_batch(layer):
+    """A decode batch of 4 tokens, top-8 of 128 experts: 32 routed rows,
+    some experts with 2-3 of them; AUTO takes the GEMV (P <= 4 E)."""
+    off, r2t = synth.uniform_routing(4, layer.E, 8, seed=93)
+    assert np.diff(off).max() >= 2
+    if layer is synth.QWEN_GATE_UP:
+        _full_check("nf4", layer.E, layer.N, layer.K, layer.w_std, off, r2t, 4, "auto")
+    else:
+        _full_check("nf4", layer.E, layer.N, layer.K, layer.w_std, off, None, 32, "auto")
 
 
 def _sampled_check(fmt, layer, off, r2t, T, mode, nrows, seed):
