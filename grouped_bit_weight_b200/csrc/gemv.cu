@@ -6,7 +6,8 @@
 // routed row per expert every weight byte is used once, so the kernel is
 // bound by HBM and never touches the tensor cores.
 //
-// B200 design (one CTA of 12 warps per SM):
+// B200 design (two CTAs of 8 warps per SM, 128 registers a thread; a warp's
+// share of a decode-sized launch fits one round of loads):
 //   work   the P*N weight rows (routed row p, output column n) are cut into
 //          row groups of RG rows (G lanes per row, RG = 32 / G); each CTA
 //          takes a contiguous range of groups and each warp a contiguous
@@ -50,7 +51,7 @@
 namespace gbw {
 namespace {
 
-constexpr int kThreads = 384;  // 12 warps: up to 168 registers a thread
+constexpr int kThreads = 256;  // 8 warps, <= 128 registers: two CTAs per SM
 constexpr int kWarps = kThreads / 32;
 constexpr int kLutBytes = 256 * 256;  // 256 entries x 256-byte rows (lanes use 128 bytes)
 // Shared-window offset of the dynamic shared memory of a kernel without
@@ -131,10 +132,11 @@ __device__ __forceinline__ float dot_unit(const uint4& q, const uint32_t (&x)[16
   return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
-// Row groups a warp loads per round (register budget for codes + scales).
-template <int UPL>
+// Row groups a warp loads per round (register budget for codes + scales,
+// within 128 registers a thread).
+template <Fmt F, int UPL>
 struct Round {
-  static constexpr int MG = UPL == 1 ? 12 : (UPL == 2 ? 7 : 5);
+  static constexpr int MG = UPL == 1 ? 10 : (UPL == 2 ? 6 : (F == Fmt::NF4 ? 2 : 3));
 };
 
 // The row groups [g0, g1) of one warp, after the kernel's prologue.
@@ -145,7 +147,7 @@ __device__ __forceinline__ void gemv_main(const GroupedProblem& pb, const int32_
   static_assert(!kGLU || G == 32, "the SwiGLU variant takes one row per group");
   constexpr int RG = 32 / G;                // rows per row group
   // row groups per load round (even for SwiGLU: gate/up pairs)
-  constexpr int MG = kGLU ? (Round<UPL>::MG & ~1) : Round<UPL>::MG;
+  constexpr int MG = kGLU ? (Round<F, UPL>::MG & ~1) : Round<F, UPL>::MG;
   const int lane = threadIdx.x & 31;
   const int li = lane % G, rs = lane / G;
   const int64_t K = pb.K, N = pb.N;
@@ -274,7 +276,7 @@ __device__ __forceinline__ void gemv_main(const GroupedProblem& pb, const int32_
 }
 
 template <Fmt F, int G, int UPL, bool kGLU>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);  // the table: 256 rows of 256 bytes
@@ -311,8 +313,8 @@ gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
   // writes its 128-byte row with eight 16-byte stores, starting at chunk
   // b % 8 so the 32 stores of a warp instruction spread over all banks.  It
   // touches no caller memory.
-  if (threadIdx.x < 256) {
-    const uint32_t b = threadIdx.x;
+  {
+    const uint32_t b = threadIdx.x;  // 256 threads: one entry each
     const uint32_t qe = (F == Fmt::NF4) ? (b >> 4) : (b & 15u);
     const uint32_t qo = (F == Fmt::NF4) ? (b & 15u) : (b >> 4);
     const uint32_t v =
@@ -417,7 +419,7 @@ cudaError_t launch_gemv(Fmt f, const GroupedProblem& pb, int num_sms,
   const int64_t ngroups = pb.P * (pb.N / (32 / sh.G));
   // the kernel keys its activation rows as token * npass + pass in 32 bits
   if ((int64_t)std::max<int64_t>(pb.T, pb.P) * sh.npass >= INT32_MAX) return cudaErrorInvalidValue;
-  const int grid = (int)std::min<int64_t>(num_sms, (ngroups / (glu ? 2 : 1) + kWarps - 1) / kWarps);
+  const int grid = (int)std::min<int64_t>(2 * num_sms, (ngroups / (glu ? 2 : 1) + kWarps - 1) / kWarps);
   if (glu) {
 #define GBW_GEMV_GLU(FF)                                                              \
   switch (sh.UPL) {                                                                   \
