@@ -282,13 +282,16 @@ def run_ours(args, rank, world, dev):
             for _ in range(reps):
                 g.replay()
 
-    run_graphs(warm_graphs)
-    torch.cuda.synchronize()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
+    # The clock sampler starts before the warm-up (it needs a moment to come
+    # up), so the warm-up runs right before the timed region and the GPU is
+    # not left idle between them.
     with Clocks(dev.index if dev.index is not None else 0) as clk:
+        run_graphs(warm_graphs)
+        torch.cuda.synchronize()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
