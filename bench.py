@@ -547,9 +547,12 @@ def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):
         d_off, d_r2t = torch.from_numpy(off).to(dev), torch.from_numpy(r2t).to(dev)
         x = torch.randn((2048, L.K), generator=gen, device=dev).to(torch.bfloat16)
         o = torch.empty((P, L.N), dtype=torch.bfloat16, device=dev)
-        out.append(tc_entry(f"gpt-oss-20b {L.name.split('_')[-1]} MXFP4 batch 2048 (P=8192, N={L.N}, K={L.K})",
-                            gemm_flops(P, L.N, L.K),
-                            lambda: gbw.gmxfp4_grouped_gemm(x, w[0], w[1], d_off, d_r2t, out=o)))
+        packed = tc_entry(f"gpt-oss-20b {L.name.split('_')[-1]} MXFP4 batch 2048 (P=8192, N={L.N}, K={L.K})",
+                          gemm_flops(P, L.N, L.K),
+                          lambda: gbw.gmxfp4_grouped_gemm(x, w[0], w[1], d_off, d_r2t, out=o))
+        out.append(packed)
+        out.append(comparator_prefill(torch, gbw.gmxfp4_dequant, w, L, x, off, d_r2t, packed,
+                                      graph_ms, dev, "gpt-oss-20b batch 2048"))
         dyg = (torch.randn((P, L.N), generator=gen, device=dev) * 1e-2).to(torch.bfloat16)
         dxg = torch.empty((P, L.K), dtype=torch.bfloat16, device=dev)
         out.append(tc_entry(f"gpt-oss-20b {L.name.split('_')[-1]} MXFP4 dgrad batch 2048 (P=8192, N={L.N}, K={L.K})",
@@ -582,43 +585,49 @@ def secondary(torch, gbw, synth, gen, dev, stream, hbm, bf16, peak_kind):
     return out
 
 
+def comparator_prefill(torch, dequant, w, L, xin, off, d_r2t, packed, graph_ms, dev, what):
+    """Dequantise-then-GEMM for one projection of a large batch: every
+    expert of the layer decoded to bf16 in one launch, the routed rows
+    gathered (index_select through row_to_token, when given), one cuBLAS
+    bf16 matmul per expert with rows; one CUDA graph, timed by replays."""
+    live = [int(e) for e in np.nonzero(np.diff(off))[0]]
+    P = int(off[-1])
+    wbf = torch.empty((L.E, L.N, L.K), dtype=torch.bfloat16, device=dev)
+    xg = torch.empty((P, L.K), dtype=torch.bfloat16, device=dev) if d_r2t is not None else None
+    ob = torch.empty((P, L.N), dtype=torch.bfloat16, device=dev)
+    r2t_long = d_r2t.long() if d_r2t is not None else None
+
+    def step():
+        dequant(w[0], w[1], out=wbf)
+        src = xin
+        if r2t_long is not None:
+            torch.index_select(xin, 0, r2t_long, out=xg)
+            src = xg
+        for e in live:
+            a, b = int(off[e]), int(off[e + 1])
+            torch.mm(src[a:b], wbf[e].t(), out=ob[a:b])
+    ms = graph_ms(step, 1, replays=10)
+    del wbf, xg, ob
+    return {"workload": f"comparator: dequantise-then-GEMM {what} {L.name.split('_')[-1]} "
+                        f"({dequant.__name__} of all {L.E} experts + {len(live)} cuBLAS bf16 "
+                        f"matmuls)",
+            "value": round(ms, 4), "unit": "ms", "higher_is_better": False,
+            "packed_ms": packed["ms"], "packed_speedup": round(ms / packed["ms"], 3)}
+
+
 def dequant_comparator(torch, gbw, x, xd, wgu, wdn, off, r2t, d_r2t, sets, gu_prefill,
                        dn_prefill, graph_ms, dev):
     """The pages' control experiment ("dequant tax"): the same projections
     computed by first decoding the packed weights to bf16 in HBM
-    (gnf4_dequant, bit-exact), then bf16 matmuls by cuBLAS (torch.mm per
+    (gnf4_dequant or gmxfp4_dequant, bit-exact), then bf16 matmuls by cuBLAS (torch.mm per
     expert with routed rows, captured in one CUDA graph).  Reported next to
     the packed path as time and the packed path's speedup."""
     import synth
     GU, DN = synth.QWEN_GATE_UP, synth.QWEN_DOWN
-    res = []
-    cnt = np.diff(off)
-    live = [int(e) for e in np.nonzero(cnt)[0]]
-    P = int(off[-1])
-    # prefill: dequantise every expert of the layer (one launch), gather the
-    # routed rows, one matmul per expert with rows
-    r2t_long = d_r2t.long()
-    for L, w, xin, gathered, packed in ((GU, wgu, x, True, gu_prefill),
-                                        (DN, wdn, xd, False, dn_prefill)):
-        wbf = torch.empty((L.E, L.N, L.K), dtype=torch.bfloat16, device=dev)
-        xg = torch.empty((P, L.K), dtype=torch.bfloat16, device=dev)
-        ob = torch.empty((P, L.N), dtype=torch.bfloat16, device=dev)
-
-        def step():
-            gbw.gnf4_dequant(w[0], w[1], out=wbf)
-            src = xin
-            if gathered:
-                torch.index_select(xin, 0, r2t_long, out=xg)
-                src = xg
-            for e in live:
-                a, b = int(off[e]), int(off[e + 1])
-                torch.mm(src[a:b], wbf[e].t(), out=ob[a:b])
-        ms = graph_ms(step, 1, replays=10)
-        res.append({"workload": f"comparator: dequantise-then-GEMM qwen3 prefill {L.name.split('_')[-1]} "
-                                f"(gnf4_dequant of all {L.E} experts + {len(live)} cuBLAS bf16 matmuls)",
-                    "value": round(ms, 4), "unit": "ms", "higher_is_better": False,
-                    "packed_ms": packed["ms"], "packed_speedup": round(ms / packed["ms"], 3)})
-        del wbf, xg, ob
+    res = [comparator_prefill(torch, gbw.gnf4_dequant, w, L, xin, off, rows, packed, graph_ms,
+                              dev, "qwen3 prefill")
+           for L, w, xin, rows, packed in ((GU, wgu, x, d_r2t, gu_prefill),
+                                           (DN, wdn, xd, None, dn_prefill))]
     # decode layer: dequantise the 8 active experts of each projection, then
     # batched matmuls (one token for gate_up, one row per expert for down)
     wg8 = torch.empty((8, GU.N, GU.K), dtype=torch.bfloat16, device=dev)

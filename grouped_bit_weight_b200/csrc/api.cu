@@ -122,8 +122,6 @@ gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
     return fail(GBW_ERR_ALIGN, "MXFP4 scales must be 2-byte aligned");
   if (!aligned4(offsets) || (row_to_token && !aligned4(row_to_token)))
     return fail(GBW_ERR_ALIGN, "offsets / row_to_token must be 4-byte aligned");
-  if (mode == GBW_MODE_GEMM && K % 64)
-    return fail(GBW_ERR_SHAPE, "the tensor-core path needs K % 64 == 0");
   int* err = nullptr;
   int sms = 0;
   gbw_status st = device_state(&err, &sms);
@@ -133,15 +131,13 @@ gbw_status grouped_forward(Fmt f, const uint16_t* x, int64_t T, int64_t K,
   const bool fits = gemv_fits(f, pb, sms);
   if (mode == GBW_MODE_GEMV && !fits)
     return fail(GBW_ERR_SHAPE, "rows too long for the GEMV's shared-memory ring");
-  if (!fits && K % 64)
-    return fail(GBW_ERR_SHAPE, "rows too long for the GEMV and K % 64 != 0");
   // AUTO: the bandwidth GEMV while experts average at most four routed rows
   // (it streams each active expert's weights once and beats the tensor-core
   // GEMM there: measured on B200 at Qwen3-30B-A3B shapes, the GEMM wins from
-  // about six rows per expert), and for K % 64 != 0, which the GEMM's 64-wide
-  // K stages do not take
+  // about six rows per expert); the GEMM takes K % 64 == 32 (MXFP4) with a
+  // half last stage
   const bool gemv = mode == GBW_MODE_GEMV ||
-                    (mode == GBW_MODE_AUTO && fits && (P <= 4 * (int64_t)E || K % 64));
+                    (mode == GBW_MODE_AUTO && fits && P <= 4 * (int64_t)E);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = gemv ? launch_gemv(f, pb, sms, s) : launch_gemm(f, pb, sms, s);
   return e == cudaSuccess ? GBW_OK : launch_error(e);

@@ -204,6 +204,14 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src)
                : "memory");
 }
+// The same copy with `src_bytes` (0..16) read and the rest of the 16 bytes
+// zero-filled; with src_bytes == 0 nothing is read from src.
+__device__ __forceinline__ void cp_async_16_fill(uint32_t dst, const void* src,
+                                                 uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }

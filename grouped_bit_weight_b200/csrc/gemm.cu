@@ -185,7 +185,15 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t E = pb.E;
   const int64_t K = pb.K, N = pb.N;
-  const int NK = (int)(K / BK);
+  // K % 64 == 32 (plain MXFP4 matmuls only; NF4 and the SwiGLU tiles need
+  // K % 64 == 0): the last stage is half a stage.  Its upper 32 K are zeros
+  // on both sides -- activations by the TMA's out-of-range fill or a
+  // zero-filling gather copy, packed weights by the TMA's fill (code 0,
+  // decoded with scale 2^0 to +0) -- so they add nothing to the sums.  The
+  // other kernels compile without the tail code: the gather warps' loop
+  // bounds the gathered path and is kept minimal.
+  constexpr bool kTail = F == Fmt::MXFP4 && !kGLU;
+  const int NK = kTail ? (int)((K + BK - 1) / BK) : (int)(K / BK);
   const int32_t ntn = kGLU ? glu_i / NS : (int32_t)((N + BM - 1) / BM);
   const int64_t ON = kGLU ? (int64_t)glu_i : N;  // columns of out
   const bool gathered = pb.row_to_token != nullptr;
@@ -282,11 +290,18 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(&x_empty[s], ph ^ 1u, abort, pb.err)))) break;
           const uint32_t dst = smem_u32(smem + Smem::x + s * kXStageBytes);
           const uint16_t* xk = pb.x + kb * BK + chunk * 8;
+          if (!kTail || kb * BK + chunk * 8 < K) {
 #pragma unroll
-          for (int i = 0; i < kRows; ++i) {
-            const int r = r0 + 12 * i;
-            if (tk[i] >= 0)
-              cp_async_16(dst + r * 128 + ((chunk ^ (r & 7)) << 4), xk + (int64_t)tk[i] * K);
+            for (int i = 0; i < kRows; ++i) {
+              const int r = r0 + 12 * i;
+              if (tk[i] >= 0)
+                cp_async_16(dst + r * 128 + ((chunk ^ (r & 7)) << 4), xk + (int64_t)tk[i] * K);
+            }
+          } else {  // past the row's end in a half last stage: zeros
+            for (int i = 0; i < kRows; ++i) {
+              const int r = r0 + 12 * i;
+              if (tk[i] >= 0) cp_async_16_fill(dst + r * 128 + ((chunk ^ (r & 7)) << 4), pb.x, 0u);
+            }
           }
           cp_async_arrive_noinc(&x_full[s]);
         }
@@ -456,10 +471,16 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
       uint32_t v = 0;
       if (hh < nh) {
         if (lrow) {
-          if (F == Fmt::NF4)
+          if (F == Fmt::NF4) {
             v = __ldg(reinterpret_cast<const uint32_t*>(lrow + lc.kb * sbytes));
-          else
+          } else if (!kTail || !(srow & 1)) {
             v = __ldg(reinterpret_cast<const uint16_t*>(lrow + lc.kb * sbytes));
+          } else {
+            // odd rows of scales (K % 64 == 32): byte loads, and the half
+            // stage past the row's end decodes with scale byte 127 (2^0)
+            const uint8_t* p = lrow + lc.kb * sbytes;
+            v = (uint32_t)__ldg(p) | (lc.kb + 1 < NK ? (uint32_t)__ldg(p + 1) << 8 : 127u << 8);
+          }
         }
         if (step(lc) && hh + 1 < nh) lrow = lrow_of(lc.tl);
       }
@@ -747,9 +768,10 @@ cudaError_t launch_gemm(Fmt f, const GroupedProblem& pb, int num_sms,
   // at least two stages per tile (so both decode groups take part in every
   // tile) and every copy stays 16-byte aligned: rows start at multiples of
   // 64, so N * srow, glu_i * srow and the array's address must be multiples
-  // of 16.
+  // of 16; srow must be even, since the decode reads two MXFP4 scale bytes as
+  // one 16-bit word (K % 64 == 32 leaves it odd: per-thread byte loads).
   const int srow = (f == Fmt::NF4) ? (int)(pb.K / 64) * 4 : (int)(pb.K / 32);
-  const int tile_scales = (pb.K / BK >= 2) && (BM * srow <= kScaleBuf) &&
+  const int tile_scales = (pb.K / BK >= 2) && (BM * srow <= kScaleBuf) && (srow % 2 == 0) &&
                           ((pb.N * srow) % 16 == 0) && ((64 * (int64_t)srow) % 16 == 0) &&
                           ((glu_i * srow) % 16 == 0) &&
                           (reinterpret_cast<uintptr_t>(pb.scale) % 16 == 0);

@@ -53,8 +53,7 @@ typedef enum {
 
 typedef enum {
   GBW_MODE_AUTO = 0, /* GEMV when P <= 4 * E (at most ~4 routed rows per
-                        expert on average) or K % 64 != 0, else the
-                        tensor-core GEMM */
+                        expert on average), else the tensor-core GEMM */
   GBW_MODE_GEMM = 1, /* force the tcgen05 grouped GEMM */
   GBW_MODE_GEMV = 2  /* force the bandwidth GEMV (no tensor cores) */
 } gbw_mode;
@@ -107,7 +106,9 @@ GBW_API gbw_status gnf4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
  *   blocks [E, N, K/32, 16] uint8 (= [E, N, K/2]): byte j holds elements 2j
  *          (LOW nibble) and 2j+1 (high nibble); bit 3 of a code is its sign
  *   scales [E, N, K/32] uint8, e8m0 (0xFF is NaN), 2-byte aligned
- * Everything else as gnf4_grouped_gemm; requires K % 32 == 0, N % 8 == 0. */
+ * Everything else as gnf4_grouped_gemm; requires K % 32 == 0, N % 8 == 0.
+ * K % 64 == 32 is taken by both paths: the tensor-core GEMM runs its last
+ * 64-wide K stage half full, zeros in the upper half on both operands. */
 GBW_API gbw_status gmxfp4_grouped_gemm(const uint16_t* x, int64_t T, int64_t K,
                                const uint8_t* blocks, const uint8_t* scales,
                                int32_t E, int64_t N,

@@ -67,7 +67,7 @@ def test_host_validation_needs_no_gpu(fn):
     if fn == "gnf4_grouped_gemm":
         assert _call(fn, K=96) == SHAPE
     else:
-        assert _call(fn, K=96, mode=1) == SHAPE  # tensor cores need K % 64
+        assert _call(fn, K=80, mode=1) == SHAPE  # MXFP4 needs K % 32
 
 
 def test_dgrad_and_codec_validation():

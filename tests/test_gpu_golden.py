@@ -1,6 +1,7 @@
 """The hand-derived grouped-matmul cases of tests/golden/hand_worked.json on
 the GPU, through both paths: every output is exact in bf16, so the tensor
-core GEMM and the bandwidth GEMV must reproduce it bit for bit."""
+core GEMM and the bandwidth GEMV must reproduce it bit for bit.  The MXFP4
+case has K = 32: on the GEMM that is one half-full 64-wide stage."""
 import numpy as np
 import pytest
 
@@ -19,8 +20,6 @@ import synth  # noqa: E402
 def test_hand_worked_cases_exact(fmt, mode):
     import torch
     c = hand_case(fmt)
-    if mode == "gemm" and c["K"] % 64:
-        pytest.skip("the tensor-core path needs K % 64 == 0")
     fn = gbw.gnf4_grouped_gemm if fmt == "nf4" else gbw.gmxfp4_grouped_gemm
     # the library takes N % 8 == 0: pad each expert with rows whose codes all
     # decode to zero (NF4 code 7, MXFP4 code 0), which must come out as 0
