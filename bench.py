@@ -294,6 +294,12 @@ def run_ours(args, rank, world, dev):
         torch.cuda.synchronize()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
+        # a ~100 us device-side delay ahead of the start event keeps the GPU
+        # busy while the host enqueues the event and the timed graphs, so the
+        # region starts with the first kernel, not with the host's launch
+        # latency (which is tens of microseconds against a 20-step region of
+        # a few hundred)
+        torch.cuda._sleep(200_000)
         t0.record(stream)
         run_graphs(timed_graphs)
         t1.record(stream)
