@@ -362,22 +362,37 @@ Shape pick_shape(int64_t U) {
 // Dynamic shared memory: the 64 KB table, then the offsets.
 size_t gemv_smem(int32_t E) { return (size_t)kLutBytes + 4 * (size_t)(E + 1); }
 
+// Per-device, per-kernel opt-in to the kernel's dynamic shared memory.
+// Guarded by a mutex: host threads may launch concurrently.
+cudaError_t opt_in(const void* fn, size_t smem) {
+  struct Entry { const void* fn; int dev; size_t smem; };
+  static std::mutex mu;
+  static Entry done[256];
+  static int ndone = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < ndone; ++i)
+    if (done[i].fn == fn && done[i].dev == dev && done[i].smem >= smem) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  for (int i = 0; i < ndone; ++i)
+    if (done[i].fn == fn && done[i].dev == dev) {
+      done[i].smem = smem;
+      return cudaSuccess;
+    }
+  if (ndone < 256) done[ndone++] = Entry{fn, dev, smem};
+  return cudaSuccess;
+}
+
 template <Fmt F, int G, int UPL, bool kGLU = false>
 cudaError_t launch_t(const GroupedProblem& pb, int64_t ngroups, int npass,
                      int grid, cudaStream_t s) {
   auto k = gemv_kernel<F, G, UPL, kGLU>;
   const size_t smem = gemv_smem(pb.E);
-  // the shared-memory opt-in is set once per device and size
-  static size_t opted[64];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = opt_in(reinterpret_cast<const void*>(k), smem);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (opted[dev] < smem) {
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    opted[dev] = smem;
-  }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
