@@ -61,32 +61,26 @@ constexpr int kLutBytes = 256 * 256;  // 256 entries x 256-byte rows (lanes use 
 constexpr uint32_t kLutBaseGuess = 1024;
 constexpr uint32_t kRuntimeBase = 0xFFFFFFFFu;
 
-// Codebook value of code q, from immediates (a select tree, no memory
-// access: a table in constant memory costs a cold miss on every launch).
-// NF4: the 16 QLoRA levels; MXFP4: OCP e2m1 (bit 3 = sign).
-__device__ __forceinline__ float code_value(Fmt F, uint32_t q) {
-  if (F == Fmt::NF4) {
-    const float lo8[8] = {-1.0f, -0.6961928009986877f, -0.5250730514526367f,
-                          -0.39491748809814453f, -0.28444138169288635f,
-                          -0.18477343022823334f, -0.09105003625154495f, 0.0f};
-    const float hi8[8] = {0.07958029955625534f, 0.16093020141124725f,
-                          0.24611230194568634f, 0.33791524171829224f,
-                          0.44070982933044434f, 0.5626170039176941f,
-                          0.7229568362236023f, 1.0f};
-    float r = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      r = (q == (uint32_t)i) ? lo8[i] : r;
-      r = (q == (uint32_t)(i + 8)) ? hi8[i] : r;
-    }
-    return r;
-  }
-  const uint32_t m = q & 7u;
-  // e2m1 magnitude: exponent field m >> 1 (bias 1), mantissa bit m & 1
-  const float mag = (m < 2u) ? 0.5f * (float)m
-                             : __int_as_float((int)((126u + (m >> 1)) << 23)) *
-                                   (1.0f + 0.5f * (float)(m & 1u));
-  return (q & 8u) ? -mag : mag;
+// bf16 bits of the codebook value of code q, from immediates (a select
+// tree on the bits of q, no memory access: a table in constant memory costs
+// a cold miss on every launch).  Word j holds the values of codes 2j (low
+// half) and 2j + 1.  NF4: bf16_rn of the 16 QLoRA levels (-1, -0.6961928,
+// -0.5250731, -0.3949175, -0.2844414, -0.1847734, -0.0910500, 0, 0.0795803,
+// 0.1609302, 0.2461123, 0.3379152, 0.4407098, 0.5626170, 0.7229568, 1);
+// MXFP4: the e2m1 values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives
+// (bit 3 = sign, code 8 = -0), exact in bf16.
+__device__ __forceinline__ uint32_t code_bf16(Fmt F, uint32_t q) {
+  const bool nf4 = F == Fmt::NF4;
+  const uint32_t w0 = nf4 ? 0xbf32bf80u : 0x3f000000u, w1 = nf4 ? 0xbecabf06u : 0x3fc03f80u;
+  const uint32_t w2 = nf4 ? 0xbe3dbe92u : 0x40404000u, w3 = nf4 ? 0x0000bdbau : 0x40c04080u;
+  const uint32_t w4 = nf4 ? 0x3e253da3u : 0xbf008000u, w5 = nf4 ? 0x3ead3e7cu : 0xbfc0bf80u;
+  const uint32_t w6 = nf4 ? 0x3f103ee2u : 0xc040c000u, w7 = nf4 ? 0x3f803f39u : 0xc0c0c080u;
+  const uint32_t j = q >> 1;
+  const uint32_t a = (j & 1u) ? w1 : w0, b = (j & 1u) ? w3 : w2;
+  const uint32_t c = (j & 1u) ? w5 : w4, d = (j & 1u) ? w7 : w6;
+  const uint32_t e = (j & 2u) ? b : a, f = (j & 2u) ? d : c;
+  const uint32_t w = (j & 4u) ? f : e;
+  return (q & 1u) ? (w >> 16) : (w & 0xFFFFu);
 }
 
 __device__ __forceinline__ float e8m0_f32(uint32_t s) {
@@ -124,12 +118,14 @@ template <uint32_t kBase>
 __device__ __forceinline__ float dot_unit(const uint4& q, const uint32_t (&x)[16],
                                           uint32_t lane4, uint32_t base) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  // four fp32 chains of eight FMAs; a warp's units are independent, so the
+  // chains of several units interleave
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int m = 0; m < 16; ++m)  // byte << 8 | lane * 4: the lane's column of that byte's entry
-    fma_pair(a[2 * (m & 3)], a[2 * (m & 3) + 1],
+    fma_pair(a[2 * (m & 1)], a[2 * (m & 1) + 1],
              lut_ld<kBase>(prmt(w[m >> 2], lane4, 0x7604u | ((m & 3) << 4)), base), x[m]);
-  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 // Row groups a warp loads per round (register budget for codes + scales,
@@ -317,9 +313,7 @@ gemv_kernel(const GroupedProblem pb, const int64_t ngroups, const int npass) {
     const uint32_t b = threadIdx.x;  // 256 threads: one entry each
     const uint32_t qe = (F == Fmt::NF4) ? (b >> 4) : (b & 15u);
     const uint32_t qo = (F == Fmt::NF4) ? (b & 15u) : (b >> 4);
-    const uint32_t v =
-        (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qe))) |
-        ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(code_value(F, qo))) << 16);
+    const uint32_t v = code_bf16(F, qe) | (code_bf16(F, qo) << 16);
     uint8_t* row = smem_raw + b * 256;
 #pragma unroll
     for (int c = 0; c < 8; ++c)
