@@ -440,6 +440,9 @@ def measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step, world
         gbw.gnf4_grouped_gemm(d_xdn, wdn[0], wdn[1], d_off, None, out=d_odn)
         h_out.copy_(d_out, non_blocking=True)
 
+    o, r = raw[0]  # a valid routing before the first call (the buffer starts zeroed)
+    h_in_np[ao:ao + noff] = o
+    h_in_np[ar:ar + nr2t] = r
     device_part()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
@@ -472,6 +475,7 @@ def measure_e2e(torch, gbw, args, dev, stream, wgu, wdn, sets, bytes_step, world
     from_graph = h_out.clone()  # the last step's outputs, from the replayed graph
     ms_eager = timed(one)       # ends with the same step's routing
     assert torch.equal(from_graph, h_out), "graph replay and eager calls disagree"
+    assert gbw.device_status(dev) == 0, "device error during the end-to-end steps"
     del g
     return {"value": round(job_rate(bytes_step, n, world, ms_graph), 2), "unit": "GB/s",
             "eager_value": round(job_rate(bytes_step, n, world, ms_eager), 2),
