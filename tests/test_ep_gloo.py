@@ -39,27 +39,35 @@ def _bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def _topk(T: int, seed: int) -> np.ndarray:
-    """TOPK distinct experts per token, uniform."""
+def _topk(T: int, seed: int, k: int = TOPK, hot: int = -1) -> np.ndarray:
+    """k distinct experts per token, uniform; hot >= 0 sends every token's
+    first slot to expert `hot`."""
     rng = np.random.default_rng(seed)
-    return np.stack([rng.choice(E, TOPK, replace=False) for _ in range(T)]).astype(np.int64) \
-        if T else np.zeros((0, TOPK), np.int64)
+    if not T:
+        return np.zeros((0, k), np.int64)
+    ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int64)
+    if hot >= 0:
+        for t in range(T):
+            if hot in ids[t, 1:]:
+                ids[t, list(ids[t]).index(hot)] = ids[t, 0]
+            ids[t, 0] = hot
+    return ids
 
 
 def _reference(x_bits, ids, wdec):
     """The oracle's grouped forward of this rank's tokens over all experts,
     scattered to [T, k, N]."""
-    T = ids.shape[0]
+    T, k = ids.shape
     flat = ids.reshape(-1)
     order = np.argsort(flat, kind="stable")
     off = np.searchsorted(flat[order], np.arange(E + 1)).astype(np.int32)
-    out = orc.grouped_forward(x_bits, wdec, off, (order // TOPK).astype(np.int32))
-    y = np.zeros((T * TOPK, N), np.uint16)
+    out = orc.grouped_forward(x_bits, wdec, off, (order // k).astype(np.int32))
+    y = np.zeros((T * k, N), np.uint16)
     y[order] = out
-    return y.reshape(T, TOPK, N)
+    return y.reshape(T, k, N)
 
 
-def _rank(rank, world, port, tokens, q):
+def _rank(rank, world, port, tokens, q, k=TOPK, hot=-1):
     import torch.distributed as dist
 
     from grouped_bit_weight_b200.ep import ExpertParallel
@@ -72,7 +80,7 @@ def _rank(rank, world, port, tokens, q):
         T = tokens[rank]
         x_bits = synth.to_bf16_bits(synth.normal((T, K), 100 + rank)) if T else \
             np.zeros((0, K), np.uint16)
-        ids = _topk(T, 200 + rank)
+        ids = _topk(T, 200 + rank, k, hot)
         ep = ExpertParallel(E)
         e0, e1 = ep.first_expert, ep.first_expert + ep.E_local
         seen = {}
@@ -98,7 +106,7 @@ def _rank(rank, world, port, tokens, q):
         # rows this rank's experts received = routed rows of all ranks to them
         sent_here = 0
         for r in range(world):
-            ids_r = _topk(tokens[r], 200 + r)
+            ids_r = _topk(tokens[r], 200 + r, k, hot)
             sent_here += int(((ids_r >= e0) & (ids_r < e1)).sum())
         q.put((rank, bool(np.array_equal(_bits(y), ref)), tuple(y.shape),
                seen["rows"] == sent_here, seen["experts_ok"], not all(all_bad)))
@@ -106,11 +114,12 @@ def _rank(rank, world, port, tokens, q):
         dist.destroy_process_group()
 
 
-def _launch(tokens):
+def _launch(tokens, k=TOPK, hot=-1):
     world, port = len(tokens), _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, tokens, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, tokens, q, k, hot))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
@@ -118,7 +127,7 @@ def _launch(tokens):
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     got = sorted(q.get(timeout=5) for _ in range(world))
     for (rank, same, shape, rows_ok, experts_ok, control_caught), T in zip(got, tokens):
-        assert shape == (T, TOPK, N), (rank, shape)
+        assert shape == (T, k, N), (rank, shape)
         assert rows_ok and experts_ok, rank
         assert same, f"rank {rank}: expert-parallel output differs from the oracle"
         assert control_caught, "swapping a rank's experts went unnoticed"
@@ -131,6 +140,16 @@ def test_two_ranks_uneven_token_counts():
 def test_four_ranks_with_an_idle_rank():
     """Rank 2 has no tokens (it still serves its two experts)."""
     _launch([7, 19, 0, 12])
+
+
+def test_two_ranks_top1_routing():
+    _launch([6, 17], k=1)
+
+
+def test_every_token_sends_its_first_slot_to_one_expert():
+    """Expert 7 (the last rank's) receives a row from every token of every
+    rank; the other slots stay uniform."""
+    _launch([9, 4], k=3, hot=7)
 
 
 def test_single_rank_holds_every_expert_and_rejects_bad_ids():
