@@ -328,8 +328,11 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
         const uint32_t idesc0 = make_idesc_bf16(BM, wide ? (uint32_t)BH : (uint32_t)((ti.nv + 15) & ~15), 0, 0);
         const uint32_t idesc1 = make_idesc_bf16(BM, (uint32_t)((ti.nv - BH + 15) & ~15), 0, 0);
         if (!(ok = mbar_wait(&acc_empty[h0], acc.phase(h0) ^ 1u, abort, pb.err))) break;
-        if (wide && !(ok = mbar_wait(&acc_empty[h1], acc.phase(h1) ^ 1u, abort, pb.err))) break;
         tc_fence_after();
+        // a wide tile's second half is waited for just before its first MMA,
+        // so the first stage's MMAs into h0 run while the epilogue still
+        // drains h1
+        bool h1_free = !wide;
         const uint32_t d0 = tmem + h0 * 256u, d1 = tmem + h1 * 256u;
         for (int kb = 0; kb < NK; ++kb, ++g) {
           const uint32_t xs = g % XS, as = g % AS;
@@ -345,6 +348,11 @@ gemm_kernel(const GroupedProblem pb, const __grid_constant__ CUtensorMap tmx,
           tc_mma_ss(d0, ad + 4, bd + 4, idesc0, 1u);
           tc_mma_ss(d0, ad + 6, bd + 6, idesc0, 1u);
           if (wide) {
+            if (!h1_free) {
+              if (!(ok = mbar_wait(&acc_empty[h1], acc.phase(h1) ^ 1u, abort, pb.err))) break;
+              tc_fence_after();
+              h1_free = true;
+            }
             const uint64_t bd1 = bd + (uint64_t)(kXHalfBytes >> 4);
             tc_mma_ss(d1, ad, bd1, idesc1, kb != 0);
             tc_mma_ss(d1, ad + 2, bd1 + 2, idesc1, 1u);
